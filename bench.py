@@ -1,0 +1,476 @@
+"""Throughput of the DSA hot path (indexer -> top-k -> sparse MLA attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dsa|reference]
+                    [--workload prefill64k|decode64k|prefill8k|decode128k|tiny]
+
+One JSON line on rank 0.  A step is one dsa_forward over the whole workload
+(every stage of the path).  The default workload is the 64K-token prefill
+(e4m3 indexer); the same line carries a `decode` object for the 64K-context
+decode batch (64 sequences, lengths 4K..64K, bf16 indexer), measured the same
+way.
+
+Timing: W untimed warm-up steps, then K steps, each preceded by an L2 flush
+(a 512 MB write) outside its CUDA-event interval; barrier + synchronize
+around the timed region; the max over ranks.  Multi-GPU runs are weak
+scaling: every rank processes its own copy of the workload (independent
+sequences), no collective on the data path.
+
+`--impl reference` times the fp64 CPU oracle on the host cores (a bounded
+sample of query rows per step): the only place besides `cpu_baseline` where
+this script executes the oracle.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "DSA prefill & decode tokens/s at 64K ctx, k=2048; % of TC/HBM roofline"
+
+WORKLOADS = {
+    "tiny": 1, "prefill8k": 2, "decode64k": 3, "prefill64k": 4, "decode128k": 5,
+}
+DESCR = {
+    1: "DSA prefill, 1 x 256 tokens, fp32 indexer 4x32, k=32, MLA 8 heads 80/64 bf16",
+    2: "DSA prefill, 1 x 8192 tokens, bf16 indexer 64x128, k=2048, MLA 128 heads 576/512 bf16",
+    3: "DSA decode, 64 sequences x 1 query, cache 4K..64K (seeded), bf16 indexer 64x128, k=2048, "
+       "MLA 128 heads 576/512 bf16",
+    4: "DSA prefill, 1 x 65536 tokens, e4m3 indexer 64x128 (per-token scales), k=2048, "
+       "MLA 128 heads 576/512 bf16",
+    5: "DSA decode, 16 sequences x 1 query, cache 131072, e4m3 indexer, k=2048, MLA 128 heads "
+       "576/512 bf16",
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm": d["hbm_gbs"], "bf16": d["bf16_tflops"],
+                "bf16_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------- work model
+def algorithmic_work(wl):
+    """Per-row units of the method's own work (not the dense work it skips).
+
+    indexer: 2*H_I*D_I flop per causal (t, s) pair; key bytes D_I*esize
+             (+4 for an fp8 scale) per key a decode row scans;
+    top-k:   4 B read per candidate + 4k B written per row;
+    attention: H*(2*D_K + 2*D_V) flop and D_K*2 gathered bytes per
+             (row, selected position).
+    """
+    c = wl.cfg
+    n = (wl.tpos + 1).astype(np.float64)
+    sel = np.minimum(n, c.k)
+    esz = {"f32": 4, "bf16": 2, "e4m3": 1}[c.idx_dtype]
+    return {
+        "idx_flop": 2.0 * c.H_I * c.D_I * n,
+        "idx_bytes": n * (c.D_I * esz + (4 if c.idx_dtype == "e4m3" else 0)),
+        "topk_bytes": 4.0 * n + 4.0 * c.k,
+        "attn_flop": c.H * (2.0 * c.D_K + 2.0 * c.D_V) * sel,
+        "attn_bytes": 2.0 * c.D_K * sel,
+    }
+
+
+def slab_rows(wl):
+    """Rows per slab of dsa_forward (scores slab capped at 1 GiB)."""
+    rows = max(1, (1 << 30) // (wl.max_len * 4))
+    return min(rows, wl.n_q)
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of this GPU's SM clock and throttle reasons."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        uuid = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
+        except Exception:
+            pass
+        sel = ["-i", uuid] if uuid else []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- device run
+def run_device(cid, steps, warmup, rank, world, do_e2e=True):
+    import sparse_attention_relu_b200 as dsa
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = workloads.generate(cid, pin=do_e2e)
+    c = wl.cfg
+    d = wl.to(dev)
+    lay = dsa.Layout.of(wl, d.kv_offsets)
+    args = dsa.forward_args(q_idx=d.q_idx, q_scale=d.q_scale, w=d.w, k_idx=d.k_idx,
+                            k_scale=d.k_scale, q=d.q, kv=d.kv, D_V=c.D_V, sm_scale=c.sm_scale,
+                            k=c.k)
+    nws = dsa.dsa_forward_workspace_size(lay, args)
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+    out = torch.empty(wl.n_q, c.H, c.D_V, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(wl.n_q, c.H, dtype=torch.float32, device=dev)
+    flush = torch.empty(128 << 20, dtype=torch.float32, device=dev)  # 512 MB > L2
+    n_slab = math.ceil(wl.n_q / slab_rows(wl))
+    n_ev = 1 + 4 * n_slab + 1
+    stream = torch.cuda.current_stream()
+
+    def step(evs):
+        return dsa.dsa_forward_timed(lay, args, out, lse, None, ws, evs)
+
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    for _ in range(warmup):
+        step(evs)
+    torch.cuda.synchronize()
+    st = dsa.dsa_device_status()
+    if st != dsa.DSA_OK:
+        raise RuntimeError(f"device status after warm-up: {dsa.dsa_status_string(st)}")
+
+    step_ms, stage_ms, launches = [], {}, 0
+    sampler = ClockSampler(torch.cuda.current_device())
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(steps):
+        flush.fill_(float(i))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kinds, nl = step(evs)
+        e1.record(stream)
+        e1.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
+        launches += nl
+        for j, kd in enumerate(kinds):
+            stage_ms.setdefault(kd, []).append(evs[j].elapsed_time(evs[j + 1]))
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    ms = sum(step_ms) / steps
+    st = dsa.dsa_device_status()
+    if st != dsa.DSA_OK:
+        raise RuntimeError(f"device status after timing: {dsa.dsa_status_string(st)}")
+
+    e2e = None
+    if do_e2e:
+        e2e = run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream)
+    return wl, ms, stage_ms, launches, clocks, e2e
+
+
+def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
+    """Same metric through the public API with host buffers: every step copies
+    the step's inputs from pinned host memory and reads the result back."""
+    names = ["q_idx", "q_scale", "w", "k_idx", "k_scale", "q", "kv", "kv_offsets"]
+    host = {n: getattr(wl, n) for n in names if getattr(wl, n) is not None}
+    dbuf = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    out_h = torch.empty(wl.n_q, c.H, c.D_V, dtype=torch.bfloat16, pin_memory=True)
+    lse_h = torch.empty(wl.n_q, c.H, dtype=torch.float32, pin_memory=True)
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    lay2 = dsa.Layout.of(wl, dbuf["kv_offsets"])
+    args = dsa.forward_args(q_idx=dbuf["q_idx"], q_scale=dbuf.get("q_scale"), w=dbuf["w"],
+                            k_idx=dbuf["k_idx"], k_scale=dbuf.get("k_scale"), q=dbuf["q"],
+                            kv=dbuf["kv"], D_V=c.D_V, sm_scale=c.sm_scale, k=c.k)
+    out = torch.empty(wl.n_q, c.H, c.D_V, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(wl.n_q, c.H, dtype=torch.float32, device=dev)
+
+    def one():
+        for n, t in host.items():
+            dbuf[n].copy_(t, non_blocking=True)
+        dsa.dsa_forward(lay2, args, out, lse, None, ws)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"ms_per_step": ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def roofline(wl, stage_ms, peaks):
+    """Dominant kernel (largest share of the step) against its roofline."""
+    w = algorithmic_work(wl)
+    tot = {k: sum(v) for k, v in stage_ms.items()}
+    if not tot:
+        return None, {}
+    kind = max(tot, key=tot.get)
+    per_launch_ms = statistics.mean(stage_ms[kind])
+    c = wl.cfg
+    slabs = math.ceil(wl.n_q / slab_rows(wl))
+    # every launch of a kind processes one slab; average work per launch
+    if kind == 2:
+        work = w["attn_flop"].sum() / slabs
+        bound, unit = "tensor", "TFLOP/s"
+        achieved = work / (per_launch_ms * 1e-3) / 1e12
+        peak = peaks["bf16_sustained"]
+        if c.mode == "decode":  # gather-bound: HBM roofline of the gathered rows
+            work = w["attn_bytes"].sum() / slabs
+            bound, unit = "hbm", "GB/s"
+            achieved = work / (per_launch_ms * 1e-3) / 1e9
+            peak = peaks["hbm"]
+    elif kind == 0:
+        if c.mode == "decode":
+            work = w["idx_bytes"].sum() / slabs
+            bound, unit = "hbm", "GB/s"
+            achieved = work / (per_launch_ms * 1e-3) / 1e9
+            peak = peaks["hbm"]
+        else:
+            work = w["idx_flop"].sum() / slabs
+            bound, unit = "tensor", "TFLOP/s"
+            achieved = work / (per_launch_ms * 1e-3) / 1e12
+            peak = peaks["bf16_sustained"] * (2.0 if c.idx_dtype == "e4m3" else 1.0)
+    else:
+        work = w["topk_bytes"].sum() / slabs
+        bound, unit = "hbm", "GB/s"
+        achieved = work / (per_launch_ms * 1e-3) / 1e9
+        peak = peaks["hbm"]
+    names = {0: "indexer", 1: "topk", 2: "sparse_mla_attn", 3: "split_combine"}
+    shares = {names[k]: round(v / sum(tot.values()), 4) for k, v in tot.items()}
+    return {"kernel": names[kind], "bound": bound, "achieved": round(achieved, 2),
+            "peak": peak, "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": peaks["source"] + (" (x2 nominal fp8/bf16 ratio)" if
+                                             unit == "TFLOP/s" and kind == 0 and
+                                             c.idx_dtype == "e4m3" else ""),
+            "launch_ms": round(per_launch_ms, 4)}, shares
+
+
+# --------------------------------------------------------------- oracle runs
+def oracle_rows(wl, rows):
+    """Runs the whole oracle path (indexer, top-k, attention) on `rows`."""
+    import oracle
+
+    c = wl.cfg
+    I = oracle.indexer_scores(wl.qrow[rows], wl.kbase[rows], wl.tpos[rows], wl.raw(wl.q_idx),
+                              wl.raw(wl.w), wl.raw(wl.k_idx), dtype=c.idx_dtype, ld=wl.max_len,
+                              q_scale=wl.raw(wl.q_scale), k_scale=wl.raw(wl.k_scale))
+    idx = oracle.topk(I, wl.tpos[rows] + 1, c.k)
+    oracle.sparse_mla_attn(wl.qrow[rows], wl.kbase[rows], idx, wl.raw(wl.q), wl.raw(wl.kv),
+                           D_V=c.D_V, sm_scale=c.sm_scale)
+
+
+def cpu_baseline(cid, budget_s=20.0, wl=None):
+    """The oracle as it stands on this host's cores, over an evenly spaced
+    sample of query rows (an unbiased estimate of the per-row mean cost),
+    grown until about `budget_s` seconds of work."""
+    import oracle
+
+    oracle.build()
+    wl = wl or workloads.generate(cid)
+    n = 2
+    done_rows, t_used = 0, 0.0
+    while t_used < budget_s and done_rows < wl.n_q:
+        rows = workloads.sample_rows(wl.n_q, n)
+        t0 = time.perf_counter()
+        oracle_rows(wl, rows)
+        dt = time.perf_counter() - t0
+        done_rows, t_used = len(rows), dt
+        if dt > budget_s / 3:
+            break
+        n *= 2
+    return {"value": round(done_rows / t_used, 3), "unit": "tokens/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{done_rows} evenly spaced query rows of the same workload "
+                      f"(all three stages, fp64), {t_used:.1f} s"}
+
+
+def run_reference(cid, steps, warmup, n_gpus):
+    import oracle
+
+    oracle.build()
+    wl = workloads.generate(cid)
+    rows_per_step = 4 if wl.n_q > 4 else wl.n_q
+    offsets = np.linspace(0, wl.n_q - 1, num=max(1, (steps + warmup) * rows_per_step)).round()
+    all_rows = np.unique(offsets.astype(np.int64))
+    chunks = np.array_split(all_rows, steps + warmup)
+    for ch in chunks[:warmup]:
+        oracle_rows(wl, ch)
+    t0 = time.perf_counter()
+    done = 0
+    for ch in chunks[warmup:]:
+        oracle_rows(wl, ch)
+        done += len(ch)
+    dt = time.perf_counter() - t0
+    value = done / dt
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": n_gpus, "steps": steps, "warmup": warmup,
+            "ms_per_step": round(dt / steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": DESCR[cid], "sample_rows_per_step": rows_per_step},
+            "cpu_baseline": {"kind": "oracle", "cores": oracle.num_threads(), "value": round(value, 3),
+                             "sample": f"{done} evenly spaced query rows over {steps} steps"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
+    ap.add_argument("--workload", default="prefill64k", choices=list(WORKLOADS))
+    ap.add_argument("--decode-workload", default="decode64k", choices=list(WORKLOADS) + ["none"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cid = WORKLOADS[a.workload]
+
+    if a.impl == "reference":
+        if rank == 0:
+            run_reference(cid, a.steps, a.warmup, a.gpus)
+        return
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    peaks = load_peaks()
+    wl, ms, stage_ms, launches, clocks, e2e = run_device(cid, a.steps, a.warmup, rank, world,
+                                                         not a.no_e2e)
+    dec = None
+    if a.decode_workload != "none":
+        dcid = WORKLOADS[a.decode_workload]
+        dwl, dms, dstage, dlaunch, _, de2e = run_device(dcid, a.steps, a.warmup, rank, world,
+                                                        not a.no_e2e)
+        dec = (dwl, dms, dstage, dlaunch, de2e)
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return t.item()
+
+    ms = max_over_ranks(ms)
+    e2e_ms = max_over_ranks(e2e["ms_per_step"]) if e2e else None
+    if dec:
+        dms = max_over_ranks(dec[1])
+        de2e_ms = max_over_ranks(dec[4]["ms_per_step"]) if dec[4] else None
+    tokens = wl.n_q
+    value = world * tokens / (ms * 1e-3)
+    roof, shares = roofline(wl, stage_ms, peaks)
+    if rank == 0:
+        cfg = wl.cfg
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": {"f32": "f32", "bf16": "bf16", "e4m3": "e4m3+bf16"}[cfg.idx_dtype],
+            "data": "synthetic",
+            "config": {"workload": DESCR[cid], "tokens_per_step_per_gpu": tokens,
+                       "k": cfg.k, "l2": "flushed before every timed step (512 MB write)",
+                       "parallelism": f"{world} independent replicas (weak scaling)"},
+            "roofline": roof, "stage_share": shares,
+            "gpu_launches": launches,
+        }
+        if e2e:
+            line["e2e"] = {"value": round(world * tokens / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                           "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                           "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]}
+        if clocks:
+            line["clocks"] = clocks
+        if dec:
+            dwl = dec[0]
+            droof, dshares = roofline(dwl, dec[2], peaks)
+            line["decode"] = {"workload": DESCR[dwl.cfg.cid],
+                              "value": round(world * dwl.n_q / (dms * 1e-3), 1),
+                              "unit": "tokens/s", "ms_per_step": round(dms, 4),
+                              "roofline": droof, "stage_share": dshares,
+                              "gpu_launches": dec[3]}
+            if dec[4]:
+                line["decode"]["e2e"] = {
+                    "value": round(world * dwl.n_q / (de2e_ms * 1e-3), 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": dec[4]["h2d_bytes_per_step"],
+                    "d2h_bytes_per_step": dec[4]["d2h_bytes_per_step"]}
+        if world == 1 and not a.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cid, wl=wl)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

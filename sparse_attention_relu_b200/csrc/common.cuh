@@ -1,0 +1,96 @@
+// Internal helpers shared by the libdsa kernels (not part of the ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dsa.h"
+
+namespace dsa {
+
+// Bits of the per-device status word (see dsa_device_status).
+enum : unsigned {
+  kErrTimeout = 1u,     // a bounded wait ran out
+  kErrBadOffsets = 2u,  // kv_offsets not monotone / out of range
+  kErrBadIndex = 4u,    // an index outside [0, L_b) (other than -1)
+};
+
+// Description of the query rows, passed by value to every kernel.
+struct Rows {
+  unsigned* status;     // this device's status word (see dsa_device_status)
+  const int32_t* offs;  // [B+1] device
+  int32_t B;
+  int32_t mode;  // DSA_PREFILL / DSA_DECODE
+  int32_t max_len;
+  int32_t n_q;
+  int64_t n_k;
+};
+
+__device__ __forceinline__ void raise_status(const Rows& R, unsigned bits) {
+  atomicOr(R.status, bits);
+}
+
+struct RowInfo {
+  int64_t kbase;  // first cache row of the sequence
+  int32_t t;      // query position inside the sequence (-1: no candidates)
+  int32_t len;    // sequence length
+  int32_t seq;
+};
+
+// Locates query row r.  Offsets that break the layout contract make the row
+// empty (t = -1) and raise kErrBadOffsets.
+__device__ __forceinline__ RowInfo row_info(const Rows& R, int32_t r) {
+  RowInfo ri{0, -1, 0, 0};
+  if (R.mode == DSA_DECODE) {
+    int32_t b = r;
+    int32_t o0 = __ldg(R.offs + b), o1 = __ldg(R.offs + b + 1);
+    if (o0 < 0 || o1 < o0 || (int64_t)o1 > R.n_k || o1 - o0 > R.max_len) {
+      raise_status(R, kErrBadOffsets);
+      return ri;
+    }
+    ri.kbase = o0;
+    ri.len = o1 - o0;
+    ri.t = ri.len - 1;
+    ri.seq = b;
+    return ri;
+  }
+  // prefill: largest b with offs[b] <= r
+  int32_t lo = 0, hi = R.B - 1;
+  while (lo < hi) {
+    int32_t mid = (lo + hi + 1) >> 1;
+    if (__ldg(R.offs + mid) <= r) lo = mid; else hi = mid - 1;
+  }
+  int32_t o0 = __ldg(R.offs + lo), o1 = __ldg(R.offs + lo + 1);
+  if (o0 < 0 || o1 < o0 || r < o0 || r >= o1 || (int64_t)o1 > R.n_k || o1 - o0 > R.max_len) {
+    raise_status(R, kErrBadOffsets);
+    return ri;
+  }
+  ri.kbase = o0;
+  ri.len = o1 - o0;
+  ri.t = r - o0;
+  ri.seq = lo;
+  return ri;
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+
+// Host-side launch error helper.
+inline dsa_status_t launch_status() {
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+inline int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace dsa

@@ -1,0 +1,307 @@
+// C ABI of libdsa: argument validation and the orchestration of the stages.
+// The semantics of each call are documented in include/dsa.h.
+#include <math.h>
+
+#include "kernels.cuh"
+
+namespace dsa {
+
+namespace {
+
+// The per-device status word.  Kernels receive its device address in Rows.
+__device__ unsigned g_status = 0;
+
+unsigned* status_word() {
+  static unsigned* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    addr[dev] = (unsigned*)p;
+  }
+  return addr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks the layout; fills the device-side row description.
+dsa_status_t check_layout(const dsa_layout_t* L, Rows* R) {
+  if (!L) return DSA_ERR_INVALID_ARGUMENT;
+  if (L->mode != DSA_PREFILL && L->mode != DSA_DECODE) return DSA_ERR_INVALID_ARGUMENT;
+  if (L->batch < 0 || L->max_len < 0 || L->n_q < 0 || L->n_k < 0) return DSA_ERR_INVALID_ARGUMENT;
+  if (L->batch > 0 && (!L->kv_offsets || !aligned16(L->kv_offsets)))
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (L->n_k >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;  // int32 offsets
+  if (L->mode == DSA_PREFILL) {
+    if (L->n_q != L->n_k) return DSA_ERR_INVALID_ARGUMENT;
+  } else {
+    if (L->n_q != L->batch) return DSA_ERR_INVALID_ARGUMENT;
+  }
+  if (L->n_q > 0 && (L->batch == 0 || L->max_len == 0)) return DSA_ERR_INVALID_ARGUMENT;
+  R->status = nullptr;  // filled by device_rows() once every argument passed
+  R->offs = L->kv_offsets;
+  R->B = L->batch;
+  R->mode = L->mode;
+  R->max_len = L->max_len;
+  R->n_q = L->n_q;
+  R->n_k = L->n_k;
+  return DSA_OK;
+}
+
+// Last step before launching: the device address of the status word.
+dsa_status_t device_rows(Rows* R) {
+  R->status = status_word();
+  return R->status ? DSA_OK : DSA_ERR_CUDA;
+}
+
+bool ptr_ok(const void* p, bool needed) { return !needed || (p && aligned16(p)); }
+
+dsa_status_t check_indexer(const Rows& R, const void* q_idx, const float* q_scale,
+                           const float* w, const void* k_idx, const float* k_scale, int dtype,
+                           int H_I, int D_I) {
+  if (dtype != DSA_F32 && dtype != DSA_BF16 && dtype != DSA_E4M3) return DSA_ERR_INVALID_ARGUMENT;
+  if (H_I < 1 || D_I < 1 || H_I > 128 || D_I > 256) return DSA_ERR_INVALID_ARGUMENT;
+  if ((int64_t)H_I * D_I > 16384 && !indexer_tc_supported(dtype, H_I, D_I))
+    return DSA_ERR_UNSUPPORTED;
+  const bool rows = R.n_q > 0;
+  if (!ptr_ok(q_idx, rows) || !ptr_ok(w, rows) || !ptr_ok(k_idx, R.n_k > 0))
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (dtype == DSA_E4M3) {
+    if (!ptr_ok(q_scale, rows) || !ptr_ok(k_scale, R.n_k > 0)) return DSA_ERR_INVALID_ARGUMENT;
+  } else if (q_scale || k_scale) {
+    return DSA_ERR_INVALID_ARGUMENT;
+  }
+  // row strides of the 16-byte vector / TMA paths
+  const int esz = dtype == DSA_F32 ? 4 : dtype == DSA_BF16 ? 2 : 1;
+  if ((D_I * esz) % 16) return DSA_ERR_INVALID_ARGUMENT;
+  return DSA_OK;
+}
+
+dsa_status_t check_attn(const Rows& R, const void* q, const void* kv, int k, int H, int D_K,
+                        int D_V, float sm_scale, const void* out, const float* lse) {
+  if (k < 1 || k > 16384) return DSA_ERR_INVALID_ARGUMENT;
+  if (H < 1 || H > 128 || D_K < 8 || D_K > 1024 || D_K % 8 || D_V < 8 || D_V > D_K || D_V % 8)
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!isfinite(sm_scale)) return DSA_ERR_INVALID_ARGUMENT;
+  const bool rows = R.n_q > 0;
+  if (!ptr_ok(q, rows) || !ptr_ok(kv, R.n_k > 0) || !ptr_ok(out, rows))
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (lse && !aligned16(lse)) return DSA_ERR_INVALID_ARGUMENT;
+  return DSA_OK;
+}
+
+dsa_status_t run_indexer(const Rows& R, int32_t row0, int32_t nrows, int dtype, int H_I, int D_I,
+                         const void* q_idx, const float* q_scale, const float* w,
+                         const void* k_idx, const float* k_scale, float* scores, bool fill,
+                         cudaStream_t st) {
+  if (indexer_tc_supported(dtype, H_I, D_I))
+    return launch_indexer_tc(R, row0, nrows, dtype, H_I, D_I, q_idx, q_scale, w, k_idx, k_scale,
+                             scores, R.max_len, fill, st);
+  return launch_indexer_simt(R, row0, nrows, dtype, H_I, D_I, q_idx, q_scale, w, k_idx, k_scale,
+                             scores, R.max_len, fill, st);
+}
+
+size_t attn_ws(int32_t nrows, int k, int H, int D_K, int D_V) {
+  return attn_tc_supported(H, D_K, D_V) ? attn_tc_workspace(nrows, k, H, D_V) : 0;
+}
+
+dsa_status_t run_attn(const Rows& R, int32_t row0, int32_t nrows, const void* q, const void* kv,
+                      const int32_t* idx, int k, int H, int D_K, int D_V, float sm_scale,
+                      void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (attn_tc_supported(H, D_K, D_V))
+    return launch_attn_tc(R, row0, nrows, (const uint16_t*)q, (const uint16_t*)kv, idx, k,
+                          sm_scale, (uint16_t*)out, lse, ws, ws_bytes, st);
+  return launch_attn_simt(R, row0, nrows, (const uint16_t*)q, (const uint16_t*)kv, idx, k, H, D_K,
+                          D_V, sm_scale, (uint16_t*)out, lse, st);
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Prefill slabs hold at most this many bytes of scores.
+constexpr size_t kSlabBytes = size_t(1) << 30;
+
+int32_t slab_rows(const Rows& R) {
+  if (R.n_q == 0) return 0;
+  size_t row_bytes = (size_t)R.max_len * 4;
+  size_t rows = kSlabBytes / (row_bytes ? row_bytes : 1);
+  if (rows < 1) rows = 1;
+  if (rows > (size_t)R.n_q) rows = R.n_q;
+  return (int32_t)rows;
+}
+
+struct ForwardPlan {
+  int32_t slab;
+  size_t off_scores, off_idx, off_attn, total;
+};
+
+ForwardPlan plan_forward(const Rows& R, const dsa_forward_args_t* a, bool own_idx) {
+  ForwardPlan p{};
+  p.slab = slab_rows(R);
+  size_t o = 0;
+  p.off_scores = o;
+  o = align_up(o + (size_t)p.slab * R.max_len * 4);
+  p.off_idx = o;
+  if (own_idx) o = align_up(o + (size_t)p.slab * a->k * 4);
+  p.off_attn = o;
+  o = align_up(o + attn_ws(p.slab, a->k, a->H, a->D_K, a->D_V));
+  p.total = o;
+  return p;
+}
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+int32_t dsa_abi_version(void) { return 1; }
+
+const char* dsa_status_string(dsa_status_t s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case DSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_TIMEOUT: return "a bounded device wait ran out";
+    case DSA_ERR_DEVICE_DATA: return "device data (offsets or indices) out of range";
+  }
+  return "unknown status";
+}
+
+dsa_status_t dsa_device_status(void* stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  unsigned v = 0, zero = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof v, 0, cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (v & kErrTimeout) return DSA_ERR_TIMEOUT;
+  if (v) return DSA_ERR_DEVICE_DATA;
+  return DSA_OK;
+}
+
+dsa_status_t dsa_indexer_scores(const dsa_layout_t* layout, const void* q_idx,
+                                const float* q_scale, const float* w, const void* k_idx,
+                                const float* k_scale, int32_t dtype, int32_t H_I, int32_t D_I,
+                                float* scores, void* stream) {
+  Rows R;
+  dsa_status_t s = check_layout(layout, &R);
+  if (s) return s;
+  if ((s = check_indexer(R, q_idx, q_scale, w, k_idx, k_scale, dtype, H_I, D_I))) return s;
+  if (!ptr_ok(scores, R.n_q > 0)) return DSA_ERR_INVALID_ARGUMENT;
+  if (R.n_q == 0) return DSA_OK;
+  if ((s = device_rows(&R))) return s;
+  return run_indexer(R, 0, R.n_q, dtype, H_I, D_I, q_idx, q_scale, w, k_idx, k_scale, scores,
+                     true, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_topk(const dsa_layout_t* layout, const float* scores, int32_t k, int32_t* idx,
+                      void* stream) {
+  Rows R;
+  dsa_status_t s = check_layout(layout, &R);
+  if (s) return s;
+  if (k < 1 || k > 16384) return DSA_ERR_INVALID_ARGUMENT;
+  if (!ptr_ok(scores, R.n_q > 0) || !ptr_ok(idx, R.n_q > 0)) return DSA_ERR_INVALID_ARGUMENT;
+  if (R.n_q == 0) return DSA_OK;
+  if ((s = device_rows(&R))) return s;
+  return launch_topk(R, 0, R.n_q, scores, R.max_len, k, idx, (cudaStream_t)stream);
+}
+
+size_t dsa_sparse_mla_attn_workspace_size(const dsa_layout_t* layout, int32_t k, int32_t H,
+                                          int32_t D_K, int32_t D_V) {
+  Rows R;
+  if (check_layout(layout, &R)) return 0;
+  return attn_ws(R.n_q, k, H, D_K, D_V);
+}
+
+dsa_status_t dsa_sparse_mla_attn(const dsa_layout_t* layout, const void* q, const void* kv,
+                                 const int32_t* idx, int32_t k, int32_t H, int32_t D_K,
+                                 int32_t D_V, float sm_scale, void* out, float* lse,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+  Rows R;
+  dsa_status_t s = check_layout(layout, &R);
+  if (s) return s;
+  if ((s = check_attn(R, q, kv, k, H, D_K, D_V, sm_scale, out, lse))) return s;
+  if (!ptr_ok(idx, R.n_q > 0)) return DSA_ERR_INVALID_ARGUMENT;
+  const size_t need = attn_ws(R.n_q, k, H, D_K, D_V);
+  if (need && (!workspace || ws_bytes < need || !aligned16(workspace))) return DSA_ERR_WORKSPACE;
+  if (R.n_q == 0) return DSA_OK;
+  if ((s = device_rows(&R))) return s;
+  return run_attn(R, 0, R.n_q, q, kv, idx, k, H, D_K, D_V, sm_scale, out, lse, workspace,
+                  ws_bytes, (cudaStream_t)stream);
+}
+
+size_t dsa_forward_workspace_size(const dsa_layout_t* layout, const dsa_forward_args_t* a) {
+  Rows R;
+  if (!a || check_layout(layout, &R)) return 0;
+  return plan_forward(R, a, true).total;
+}
+
+dsa_status_t dsa_forward_timed(const dsa_layout_t* layout, const dsa_forward_args_t* a,
+                               void* out, float* lse, int32_t* idx_out, void* workspace,
+                               size_t ws_bytes, void* stream, void* const* events,
+                               int32_t n_events, int32_t* kinds, int32_t* n_launched) {
+  Rows R;
+  dsa_status_t s = check_layout(layout, &R);
+  if (s) return s;
+  if (!a) return DSA_ERR_INVALID_ARGUMENT;
+  if ((s = check_indexer(R, a->q_idx, a->q_scale, a->w, a->k_idx, a->k_scale, a->idx_dtype,
+                         a->H_I, a->D_I)))
+    return s;
+  if ((s = check_attn(R, a->q, a->kv, a->k, a->H, a->D_K, a->D_V, a->sm_scale, out, lse)))
+    return s;
+  if (idx_out && !aligned16(idx_out)) return DSA_ERR_INVALID_ARGUMENT;
+  if (n_events > 0 && !events) return DSA_ERR_INVALID_ARGUMENT;
+  const ForwardPlan p = plan_forward(R, a, idx_out == nullptr);
+  if (!workspace || ws_bytes < p.total || !aligned16(workspace)) return DSA_ERR_WORKSPACE;
+  if (n_launched) *n_launched = 0;
+  if (R.n_q == 0) return DSA_OK;
+  if ((s = device_rows(&R))) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  int32_t launched = 0;
+  auto mark = [&](int32_t kind) -> dsa_status_t {
+    if (launched + 1 < n_events &&
+        cudaEventRecord((cudaEvent_t)events[launched + 1], st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    if (kinds && launched + 1 < n_events) kinds[launched] = kind;
+    ++launched;
+    if (n_launched) *n_launched = launched;
+    return DSA_OK;
+  };
+  if (n_events > 0 && cudaEventRecord((cudaEvent_t)events[0], st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  char* ws = (char*)workspace;
+  float* scores = (float*)(ws + p.off_scores);
+  for (int32_t r0 = 0; r0 < R.n_q; r0 += p.slab) {
+    const int32_t nr = (R.n_q - r0) < p.slab ? (R.n_q - r0) : p.slab;
+    int32_t* idx = idx_out ? idx_out + (int64_t)r0 * a->k : (int32_t*)(ws + p.off_idx);
+    if ((s = run_indexer(R, r0, nr, a->idx_dtype, a->H_I, a->D_I, a->q_idx, a->q_scale, a->w,
+                         a->k_idx, a->k_scale, scores, false, st)))
+      return s;
+    if ((s = mark(0))) return s;
+    if ((s = launch_topk(R, r0, nr, scores, R.max_len, a->k, idx, st))) return s;
+    if ((s = mark(1))) return s;
+    if ((s = run_attn(R, r0, nr, a->q, a->kv, idx, a->k, a->H, a->D_K, a->D_V, a->sm_scale, out,
+                      lse, ws + p.off_attn, p.total - p.off_attn, st)))
+      return s;
+    if ((s = mark(2))) return s;
+  }
+  return DSA_OK;
+}
+
+dsa_status_t dsa_forward(const dsa_layout_t* layout, const dsa_forward_args_t* a, void* out,
+                         float* lse, int32_t* idx_out, void* workspace, size_t ws_bytes,
+                         void* stream) {
+  return dsa_forward_timed(layout, a, out, lse, idx_out, workspace, ws_bytes, stream, nullptr, 0,
+                           nullptr, nullptr);
+}
+
+}  // extern "C"

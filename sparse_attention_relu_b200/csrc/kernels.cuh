@@ -1,0 +1,42 @@
+// Internal launchers of libdsa (not part of the ABI).
+//
+// Row conventions: query-row arrays (q_idx, q_scale, w, q, out, lse) are
+// indexed by the absolute query row r; per-slab arrays (scores, idx) point
+// at the slab's first row `row0` and are indexed by r - row0.
+#pragma once
+
+#include "common.cuh"
+
+namespace dsa {
+
+// Generic indexer (any dtype, H_I * D_I <= 16384, D_I <= 256).
+dsa_status_t launch_indexer_simt(const Rows& R, int32_t row0, int32_t nrows, int dtype, int H_I,
+                                 int D_I, const void* q_idx, const float* q_scale,
+                                 const float* w, const void* k_idx, const float* k_scale,
+                                 float* scores, int64_t ld, bool fill_masked, cudaStream_t st);
+
+// Tensor-core indexer (bf16 / e4m3, H_I = 64, D_I = 128).  Returns
+// DSA_ERR_UNSUPPORTED when the shape does not fit it.
+dsa_status_t launch_indexer_tc(const Rows& R, int32_t row0, int32_t nrows, int dtype, int H_I,
+                               int D_I, const void* q_idx, const float* q_scale, const float* w,
+                               const void* k_idx, const float* k_scale, float* scores, int64_t ld,
+                               bool fill_masked, cudaStream_t st);
+bool indexer_tc_supported(int dtype, int H_I, int D_I);
+
+// Radix top-k, one CTA per row.
+dsa_status_t launch_topk(const Rows& R, int32_t row0, int32_t nrows, const float* scores,
+                         int64_t ld, int k, int32_t* idx, cudaStream_t st);
+
+// Generic sparse MLA attention (H <= 128, D_V <= D_K <= 1024, multiples of 8).
+dsa_status_t launch_attn_simt(const Rows& R, int32_t row0, int32_t nrows, const uint16_t* q,
+                              const uint16_t* kv, const int32_t* idx, int k, int H, int D_K,
+                              int D_V, float sm_scale, uint16_t* out, float* lse, cudaStream_t st);
+
+// Tensor-core sparse MLA attention (H = 128, D_K = 576, D_V = 512).
+bool attn_tc_supported(int H, int D_K, int D_V);
+size_t attn_tc_workspace(int32_t nrows, int k, int H, int D_V);
+dsa_status_t launch_attn_tc(const Rows& R, int32_t row0, int32_t nrows, const uint16_t* q,
+                            const uint16_t* kv, const int32_t* idx, int k, float sm_scale,
+                            uint16_t* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st);
+
+}  // namespace dsa

@@ -1,0 +1,83 @@
+"""The C ABI loads, exports every declared entry point and rejects bad
+arguments before touching a device (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_relu_b200 as dsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            src = open(os.path.join(inc, f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(dsa_\w+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_attention_relu_b200 import build
+
+    build.build()
+    return dsa.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert {"dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert dsa.dsa_status_string(s) and dsa.dsa_status_string(s) != "unknown status"
+    assert dsa.dsa_status_string(99) == "unknown status"
+    assert dsa.dsa_abi_version() >= 1
+
+
+def _layout(**kw):
+    d = dict(mode=0, batch=1, kv_offsets=16, max_len=8, n_q=8, n_k=8)
+    d.update(kw)
+    return dsa.dsa_layout_t(d["mode"], d["batch"], d["kv_offsets"], d["max_len"], d["n_q"],
+                            d["n_k"])
+
+
+def test_argument_validation_without_device(lib):
+    E = dsa.DSA_ERR_INVALID_ARGUMENT
+    P = 4096  # a fake, 16-byte aligned "device pointer": never dereferenced
+    assert lib.dsa_topk(None, P, 4, P, None) == E
+    L = _layout()
+    assert lib.dsa_topk(ctypes.byref(L), P, 0, P, None) == E  # k < 1
+    assert lib.dsa_topk(ctypes.byref(L), P, 16385, P, None) == E
+    assert lib.dsa_topk(ctypes.byref(L), P + 4, 4, P, None) == E  # misaligned
+    assert lib.dsa_topk(ctypes.byref(L), None, 4, P, None) == E
+    bad = _layout(n_q=7)  # prefill needs n_q == n_k
+    assert lib.dsa_topk(ctypes.byref(bad), P, 4, P, None) == E
+    bad = _layout(mode=1, batch=2, n_q=3)  # decode needs n_q == batch
+    assert lib.dsa_topk(ctypes.byref(bad), P, 4, P, None) == E
+    bad = _layout(kv_offsets=None)
+    assert lib.dsa_topk(ctypes.byref(bad), P, 4, P, None) == E
+    # indexer: dtype, head sizes, scales only with e4m3
+    assert lib.dsa_indexer_scores(ctypes.byref(L), P, None, P, P, None, 7, 4, 32, P, None) == E
+    assert lib.dsa_indexer_scores(ctypes.byref(L), P, P, P, P, P, dsa.DSA_BF16, 4, 32, P, None) == E
+    assert lib.dsa_indexer_scores(ctypes.byref(L), P, None, P, P, None, dsa.DSA_E4M3, 4, 32, P,
+                                  None) == E
+    assert lib.dsa_indexer_scores(ctypes.byref(L), P, None, P, P, None, dsa.DSA_F32, 4, 3, P,
+                                  None) == E  # row not a multiple of 16 bytes
+    # attention: shape limits
+    f = lib.dsa_sparse_mla_attn
+    assert f(ctypes.byref(L), P, P, P, 4, 129, 576, 512, 0.1, P, None, None, 0, None) == E
+    assert f(ctypes.byref(L), P, P, P, 4, 128, 576, 580, 0.1, P, None, None, 0, None) == E
+    assert f(ctypes.byref(L), P, P, P, 4, 8, 80, 64, float("nan"), P, None, None, 0, None) == E
+    # empty problems succeed without launching anything
+    empty = _layout(batch=0, kv_offsets=None, max_len=0, n_q=0, n_k=0)
+    assert lib.dsa_topk(ctypes.byref(empty), None, 4, None, None) == dsa.DSA_OK
