@@ -1,0 +1,412 @@
+// Lightning indexer on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+//   I[t, s] = sum_j w[t, j] * ReLU(<q_I[t, j, :], k_I[s, :]>),   s <= t
+//
+// ("GLM sparse attention", ReLU paragraph; "Sparse Attention Architecture
+// Evolution in LLMs", Indexer section: a small scorer that scans every
+// earlier position.)  H_I = 64 heads, D_I = 128, bf16 or fp8 e4m3 inputs.
+//
+// The contraction is a GEMM with the KEYS on M and (query, head) pairs on N:
+//   D[key, (q, j)] = <k_I[key], q_I[q, j]>        M = 128 keys, N = G * 64
+// so that one TMEM lane holds every head of one key for G queries, and the
+// ReLU + weighted head sum is a private loop per thread in the epilogue,
+// with no shuffles.  fp8 scales fold in for free: q_scale (positive) moves
+// into w, k_scale multiplies the finished sum.
+//
+// Warp roles (192 threads):
+//   warp 0     TMA producer: the query block once, then a ring of key tiles
+//   warp 1     TMEM allocator and MMA issuer (one thread)
+//   warps 2-5  epilogue: TMEM -> registers, ReLU, weighted head sum, store
+// Key tiles stream through an NK-stage shared-memory ring; accumulators
+// rotate through NS TMEM slots so the MMA of the next job overlaps the
+// epilogue of the previous one.
+//
+// Work: prefill -- a CTA owns NG*G consecutive queries of one sequence and
+// every key tile up to the last query (blocks launched heaviest first);
+// decode -- a CTA owns the single query of a sequence and a chunk of KCH keys.
+#include <cudaTypedefs.h>
+
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace dsa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kHI = 64, kDI = 128, kTileK = 128;  // heads, dims, keys per tile
+constexpr int kThreads = 192;
+constexpr int kDecodeChunk = 2048;  // keys per CTA in decode
+
+template <int DT, int G, int NG, int NK>
+struct Cfg {
+  static constexpr int ESZ = DT == DSA_BF16 ? 2 : 1;
+  static constexpr int ROWB = kDI * ESZ;          // bytes per row
+  static constexpr int KC = ROWB / 128;           // 128-byte column blocks per row
+  static constexpr int N = G * kHI;               // MMA N
+  static constexpr int QB = G * NG;               // queries per CTA
+  static constexpr int QBYTES = NG * N * ROWB;
+  static constexpr int KBYTES = kTileK * ROWB;
+  static constexpr int NS = (512 / N) > 8 ? 8 : (512 / N);  // TMEM accumulator slots
+  static constexpr int TCOLS = NS * N;
+  static constexpr int UK = DT == DSA_BF16 ? 16 : 32;       // K per MMA instruction
+  static constexpr int KSTEPS = kDI / UK;
+  static constexpr uint32_t IDESC = idesc(DT == DSA_BF16 ? 1u : 0u, 128, N);
+  // shared memory map (offsets from a 1024-aligned base)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + QBYTES;
+  static constexpr int OFF_W = OFF_K + NK * KBYTES;
+  static constexpr int OFF_BAR = OFF_W + QB * kHI * 4;
+  static constexpr int NBAR = 2 * NK + 2 * NS + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
+  static_assert(TCOLS == 512 || TCOLS == 256 || TCOLS == 128, "TMEM columns");
+};
+
+struct Work {
+  int valid;          // CTA has work
+  int64_t kbase;      // first key row of the sequence
+  int32_t len;        // sequence length
+  int32_t t0;         // local position of the first query of the block
+  int32_t nq;         // queries in the block (<= QB)
+  int32_t qrow0;      // global query row of query 0 of the block
+  int32_t kt_begin, kt_end;  // key tiles
+  int32_t qvalid_lo, qvalid_hi;  // valid query positions [lo, hi) (local)
+  int32_t fill_lo, fill_hi;      // decode: key range this CTA owns (for -inf fill)
+};
+
+template <int QB>
+__device__ Work plan_prefill(const Rows& R, int32_t row0, int32_t nrows) {
+  Work w{};
+  const int b = blockIdx.y;
+  const int32_t o0 = __ldg(R.offs + b), o1 = __ldg(R.offs + b + 1);
+  if (o0 < 0 || o1 < o0 || (int64_t)o1 > R.n_k || o1 - o0 > R.max_len) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(R, kErrBadOffsets);
+    return w;
+  }
+  const int32_t lo = max(o0, row0), hi = min(o1, row0 + nrows);
+  if (lo >= hi) return w;
+  const int32_t i0 = (lo - o0) / QB, i1 = (hi - 1 - o0) / QB;
+  if ((int32_t)blockIdx.x > i1 - i0) return w;
+  const int32_t i = i1 - (int32_t)blockIdx.x;  // heaviest block first
+  w.valid = 1;
+  w.kbase = o0;
+  w.len = o1 - o0;
+  w.t0 = i * QB;
+  w.qrow0 = o0 + w.t0;
+  w.qvalid_lo = max(w.t0, lo - o0);
+  w.qvalid_hi = min(w.t0 + QB, hi - o0);
+  w.nq = QB;
+  w.kt_begin = 0;
+  w.kt_end = (w.qvalid_hi - 1) / kTileK + 1;  // keys up to the last valid query
+  return w;
+}
+
+__device__ Work plan_decode(const Rows& R, int32_t row0) {
+  Work w{};
+  const int32_t r = row0 + blockIdx.y;
+  const RowInfo ri = row_info(R, r);
+  const int32_t c0 = blockIdx.x * kDecodeChunk;
+  w.fill_lo = c0;
+  w.fill_hi = min(c0 + kDecodeChunk, R.max_len);
+  w.len = ri.len;
+  w.qrow0 = r;
+  if (ri.t < 0 || c0 > ri.t) return w;  // nothing to score (fill only)
+  w.valid = 1;
+  w.kbase = ri.kbase;
+  w.t0 = ri.t;
+  w.nq = 1;
+  w.qvalid_lo = ri.t;
+  w.qvalid_hi = ri.t + 1;
+  w.kt_begin = c0 / kTileK;
+  w.kt_end = (min(c0 + kDecodeChunk, ri.t + 1) + kTileK - 1) / kTileK;
+  return w;
+}
+
+template <int DT, int G, int NG, int NK, bool DECODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    indexer_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                      const __grid_constant__ CUtensorMap kmap, Rows R, int32_t row0,
+                      int32_t nrows, const float* __restrict__ w, const float* __restrict__ q_scale,
+                      const float* __restrict__ k_scale, float* __restrict__ scores, int64_t ld,
+                      int fill) {
+  using C = Cfg<DT, G, NG, NK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* wq = reinterpret_cast<float*>(smem + C::OFF_W);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto k_full = [&](int i) { return bar0 + 8u * i; };
+  auto k_empty = [&](int i) { return bar0 + 8u * (NK + i); };
+  auto s_full = [&](int i) { return bar0 + 8u * (2 * NK + i); };
+  auto s_empty = [&](int i) { return bar0 + 8u * (2 * NK + C::NS + i); };
+  const uint32_t q_full = bar0 + 8u * (2 * NK + 2 * C::NS);
+  const uint32_t drain = q_full + 8u;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Work wk = DECODE ? plan_decode(R, row0) : plan_prefill<C::QB>(R, row0, nrows);
+
+  if (!wk.valid) {
+    if (DECODE && fill && wk.fill_lo < wk.fill_hi) {  // a chunk past the end of the sequence
+      float* o = scores + (int64_t)blockIdx.y * ld;
+      for (int s = wk.fill_lo + tid; s < wk.fill_hi; s += kThreads) o[s] = -INFINITY;
+    }
+    return;
+  }
+
+  if (tid == 0) {
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(k_full(i), 1);
+      mbar_init(k_empty(i), 1);
+    }
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(s_full(i), 1);
+      mbar_init(s_empty(i), 4);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + C::OFF_MISC, C::TCOLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_tiles = wk.kt_end - wk.kt_begin;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch(&qmap);
+      tma_prefetch(&kmap);
+      mbar_expect_tx(q_full, C::QBYTES);
+      for (int g = 0; g < NG; ++g)
+        for (int kc = 0; kc < C::KC; ++kc)
+          tma_load_2d(sbase + C::OFF_Q + (g * C::KC + kc) * C::N * 128, &qmap, kc * (128 / C::ESZ),
+                      (wk.qrow0 + g * G) * kHI, q_full);
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int st = j % NK;
+        if (!mbar_wait(k_empty(st), ((j / NK) & 1) ^ 1, R.status) || *abort_flag) {
+          *abort_flag = 1;
+          break;
+        }
+        mbar_expect_tx(k_full(st), C::KBYTES);
+        const int32_t krow = (int32_t)(wk.kbase + (int64_t)(wk.kt_begin + j) * kTileK);
+        for (int kc = 0; kc < C::KC; ++kc)
+          tma_load_2d(sbase + C::OFF_K + st * C::KBYTES + kc * kTileK * 128, &kmap,
+                      kc * (128 / C::ESZ), krow, k_full(st));
+        ++issued;
+      }
+      // leave no copy in flight behind us
+      for (int j = max(0, issued - NK); j < issued; ++j)
+        mbar_wait(k_full(j % NK), (j / NK) & 1, R.status);
+      mbar_wait(q_full, 0, R.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(q_full, 0, R.status);
+      int job = 0;
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int st = j % NK;
+        if (!mbar_wait(k_full(st), (j / NK) & 1, R.status) || *abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = sbase + C::OFF_K + st * C::KBYTES;
+        for (int g = 0; g < NG; ++g, ++job) {
+          const int slot = job % C::NS;
+          if (!mbar_wait(s_empty(slot), ((job / C::NS) & 1) ^ 1, R.status) || *abort_flag) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b_base = sbase + C::OFF_Q + g * C::KC * C::N * 128;
+          const uint32_t d = tmem + slot * C::N;
+#pragma unroll
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const int kc = kk / 4, sub = (kk % 4) * 32;
+            const uint64_t da = desc_sw128(a_base + kc * kTileK * 128 + sub, 1024);
+            const uint64_t db = desc_sw128(b_base + kc * C::N * 128 + sub, 1024);
+            if constexpr (DT == DSA_BF16)
+              mma_bf16(d, da, db, C::IDESC, kk > 0 ? 1u : 0u);
+            else
+              mma_e4m3(d, da, db, C::IDESC, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(s_full(slot));
+        }
+        if (!ok) break;
+        mma_commit(k_empty(st));
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        mma_commit(drain);
+        mbar_wait(drain, 0, R.status);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int et = tid - 64;           // 0..127
+    const int quad = warp & 3;         // TMEM lane quadrant this warp may read
+    for (int i = et; i < C::QB * kHI; i += 128) {
+      const int qi = i / kHI, h = i - qi * kHI;
+      const int32_t tq = wk.t0 + qi;
+      float v = 0.f;
+      if (qi < wk.nq && tq >= wk.qvalid_lo && tq < wk.qvalid_hi) {
+        const int64_t qr = wk.qrow0 + qi;
+        v = __ldg(w + qr * kHI + h);
+        if (q_scale) v *= __ldg(q_scale + qr * kHI + h);
+      }
+      wq[i] = v;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    int job = 0;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int32_t s = (wk.kt_begin + j) * kTileK + quad * 32 + lane;
+      float ks = 1.f;
+      if (DT == DSA_E4M3 && k_scale && s < wk.len) ks = __ldg(k_scale + wk.kbase + s);
+      for (int g = 0; g < NG; ++g, ++job) {
+        const int slot = job % C::NS;
+        if (!mbar_wait(s_full(slot), (job / C::NS) & 1, R.status) || *abort_flag) {
+          *abort_flag = 1;
+          j = n_tiles;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int qq = 0; qq < G; ++qq) {
+          const int qi = g * G + qq;
+          const float* wr = wq + qi * kHI;
+          const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + slot * C::N + qq * kHI;
+          float acc = 0.f;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tmem_ld32(ta + half * 32, v);
+#pragma unroll
+            for (int h = 0; h < 32; ++h) acc = fmaf(wr[half * 32 + h], fmaxf(v[h], 0.f), acc);
+          }
+          const int32_t tq = wk.t0 + qi;
+          if (tq >= wk.qvalid_lo && tq < wk.qvalid_hi && s < R.max_len) {
+            float* o = scores + (int64_t)(wk.qrow0 + qi - row0) * ld;
+            if (s <= tq)
+              o[s] = acc * ks;
+            else if (fill)
+              o[s] = -INFINITY;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_empty(slot));
+      }
+    }
+    // -inf beyond the last scored tile (unit call only)
+    if (fill) {
+      for (int qi = 0; qi < C::QB; ++qi) {
+        const int32_t tq = wk.t0 + qi;
+        if (qi >= wk.nq || tq < wk.qvalid_lo || tq >= wk.qvalid_hi) continue;
+        float* o = scores + (int64_t)(wk.qrow0 + qi - row0) * ld;
+        const int32_t from = wk.kt_end * kTileK;
+        const int32_t to = DECODE ? wk.fill_hi : R.max_len;
+        for (int s = from + et; s < to; s += 128) o[s] = -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TCOLS);
+  }
+}
+
+}  // namespace
+
+bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize,
+                  uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+      return false;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)esize};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool indexer_tc_supported(int dtype, int H_I, int D_I) {
+  return (dtype == DSA_BF16 || dtype == DSA_E4M3) && H_I == kHI && D_I == kDI;
+}
+
+template <int DT, int G, int NG, int NK, bool DECODE>
+static dsa_status_t launch_cfg(const Rows& R, int32_t row0, int32_t nrows, const void* q_idx,
+                               const float* q_scale, const float* w, const void* k_idx,
+                               const float* k_scale, float* scores, int64_t ld, bool fill,
+                               cudaStream_t st) {
+  using C = Cfg<DT, G, NG, NK>;
+  CUtensorMap qmap, kmap;
+  const CUtensorMapDataType tdt =
+      DT == DSA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const uint32_t box_cols = 128 / C::ESZ;
+  if (!make_tmap_2d(&qmap, q_idx, tdt, C::ESZ, kDI, (uint64_t)R.n_q * kHI, box_cols, C::N) ||
+      !make_tmap_2d(&kmap, k_idx, tdt, C::ESZ, kDI, (uint64_t)R.n_k, box_cols, kTileK))
+    return DSA_ERR_CUDA;
+  auto kfn = indexer_tc_kernel<DT, G, NG, NK, DECODE>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  dim3 grid;
+  if (DECODE) {
+    grid = dim3((R.max_len + kDecodeChunk - 1) / kDecodeChunk, nrows);
+  } else {
+    const int32_t span = nrows < R.max_len ? nrows : R.max_len;
+    grid = dim3((span + C::QB - 1) / C::QB + 1, R.B);
+  }
+  kfn<<<grid, kThreads, C::SMEM, st>>>(qmap, kmap, R, row0, nrows, w, q_scale, k_scale, scores,
+                                       ld, fill ? 1 : 0);
+  return launch_status();
+}
+
+dsa_status_t launch_indexer_tc(const Rows& R, int32_t row0, int32_t nrows, int dtype, int H_I,
+                               int D_I, const void* q_idx, const float* q_scale, const float* w,
+                               const void* k_idx, const float* k_scale, float* scores, int64_t ld,
+                               bool fill, cudaStream_t st) {
+  if (!indexer_tc_supported(dtype, H_I, D_I)) return DSA_ERR_UNSUPPORTED;
+  if (nrows <= 0) return DSA_OK;
+  const bool decode = R.mode == DSA_DECODE;
+  if (dtype == DSA_BF16) {
+    if (decode)
+      return launch_cfg<DSA_BF16, 1, 1, 6, true>(R, row0, nrows, q_idx, q_scale, w, k_idx,
+                                                 k_scale, scores, ld, fill, st);
+    return launch_cfg<DSA_BF16, 4, 2, 2, false>(R, row0, nrows, q_idx, q_scale, w, k_idx,
+                                                k_scale, scores, ld, fill, st);
+  }
+  if (decode)
+    return launch_cfg<DSA_E4M3, 1, 1, 8, true>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale,
+                                               scores, ld, fill, st);
+  return launch_cfg<DSA_E4M3, 4, 2, 4, false>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale,
+                                              scores, ld, fill, st);
+}
+
+}  // namespace dsa

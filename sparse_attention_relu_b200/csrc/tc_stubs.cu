@@ -1,10 +1,6 @@
-// Placeholder until the tensor-core kernels land.
+// Placeholder until the tensor-core attention kernel lands.
 #include "kernels.cuh"
 namespace dsa {
-bool indexer_tc_supported(int, int, int) { return false; }
-dsa_status_t launch_indexer_tc(const Rows&, int32_t, int32_t, int, int, int, const void*,
-                               const float*, const float*, const void*, const float*, float*,
-                               int64_t, bool, cudaStream_t) { return DSA_ERR_UNSUPPORTED; }
 bool attn_tc_supported(int, int, int) { return false; }
 size_t attn_tc_workspace(int32_t, int, int, int) { return 0; }
 dsa_status_t launch_attn_tc(const Rows&, int32_t, int32_t, const uint16_t*, const uint16_t*,
