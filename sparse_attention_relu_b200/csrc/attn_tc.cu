@@ -418,9 +418,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 4; ++e) {
           const float p0 = exp2f(s[8 * c + 2 * e] - mref);
           const float p1 = exp2f(s[8 * c + 2 * e + 1] - mref);
-          w4[e] = pack_bf16(p0, p1);
-          const __nv_bfloat162 q = *reinterpret_cast<const __nv_bfloat162*>(&w4[e]);
-          lsum += __low2float(q) + __high2float(q);
+          w4[e] = pack_bf16(p0, p1);  // bf16 only as the MMA operand
+          lsum += p0 + p1;            // the denominator keeps fp32 probabilities
         }
         *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
