@@ -143,6 +143,37 @@ dsa_status_t dsa_sparse_mla_attn(const dsa_layout_t* layout, const void* q, cons
 size_t dsa_sparse_mla_attn_workspace_size(const dsa_layout_t* layout, int32_t k, int32_t H,
                                           int32_t D_K, int32_t D_V);
 
+/*
+ * dsa_sparse_mla_attn for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it exists for the
+ * library's users.  Some callers cannot call cudaMalloc or any allocating
+ * routine: code that runs while a CUDA graph is being captured with a strict
+ * capture mode, code inside a framework whose memory pool owns the whole
+ * device, or plug-ins that are handed tensors but no allocator.  This call
+ * takes the same arguments as dsa_sparse_mla_attn minus the workspace: the
+ * decode split partials go to a fixed 64 MiB array that the library owns
+ * on every GPU where it is loaded, held until the process exits.
+ *  - Capacity: a call whose split plan needs more than 64 MiB of partials
+ *    (128 heads x 513 floats per (query row, split) pair, so at most 255
+ *    pairs) returns DSA_ERR_WORKSPACE without launching anything.  With
+ *    k <= 2048 that is every batch except 128..147 query rows; 148 rows or
+ *    more need no partials at all.  Shapes that do not run on the tensor
+ *    cores need no scratch and are never refused for size.
+ *  - Nothing needs zeroing: every call writes each partial it later reads.
+ *  - The array is shared by all calls on a device and keeps the last call's
+ *    contents: calls whose executions overlap on the GPU (different streams,
+ *    no ordering between them) race on it and must be serialised.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ * Results equal those of dsa_sparse_mla_attn on the same inputs.
+ */
+dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_layout_t* layout, const void* q,
+                                         const void* kv, const int32_t* idx, int32_t k, int32_t H,
+                                         int32_t D_K, int32_t D_V, float sm_scale, void* out,
+                                         float* lse, void* stream);
+
 /* Inputs of the whole chain (each field as in the stage calls above). */
 typedef struct {
   int32_t idx_dtype; /* dsa_dtype_t of q_idx / k_idx */

@@ -68,6 +68,8 @@ def lib():
         L.dsa_topk.argtypes = [LP, P, I32, P, P]
         L.dsa_sparse_mla_attn.argtypes = [LP, P, P, P, I32, I32, I32, I32, ctypes.c_float, P, P,
                                           P, SZ, P]
+        L.dsa_sparse_mla_attn_noalloc.argtypes = [LP, P, P, P, I32, I32, I32, I32,
+                                                  ctypes.c_float, P, P, P]
         L.dsa_sparse_mla_attn_workspace_size.argtypes = [LP, I32, I32, I32, I32]
         L.dsa_sparse_mla_attn_workspace_size.restype = SZ
         L.dsa_forward_workspace_size.argtypes = [LP, AP]
@@ -78,7 +80,8 @@ def lib():
         L.dsa_status_string.argtypes = [ctypes.c_int]
         L.dsa_status_string.restype = ctypes.c_char_p
         L.dsa_abi_version.restype = I32
-        for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward",
+        for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn",
+                     "dsa_sparse_mla_attn_noalloc", "dsa_forward",
                      "dsa_forward_timed", "dsa_device_status"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -164,6 +167,18 @@ def dsa_sparse_mla_attn(layout: Layout, q, kv, idx, k: int, D_V: int, sm_scale: 
                                      int(D_V), float(sm_scale), _ptr(out), _ptr(lse),
                                      _ptr(workspace), ws_bytes, _stream(stream)),
            "dsa_sparse_mla_attn")
+    return out
+
+
+def dsa_sparse_mla_attn_noalloc(layout: Layout, q, kv, idx, k: int, D_V: int, sm_scale: float,
+                                out, lse=None, stream=None):
+    """Stage 3 without a workspace: the library's fixed device scratch holds
+    the split partials (for callers that cannot allocate; see include/dsa.h)."""
+    _, H, D_K = q.shape
+    _check(lib().dsa_sparse_mla_attn_noalloc(layout.ref, _ptr(q), _ptr(kv), _ptr(idx), int(k), H,
+                                             D_K, int(D_V), float(sm_scale), _ptr(out), _ptr(lse),
+                                             _stream(stream)),
+           "dsa_sparse_mla_attn_noalloc")
     return out
 
 

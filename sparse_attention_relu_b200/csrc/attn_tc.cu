@@ -520,6 +520,11 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(int32_t row0, int nsp
   if (lse && threadIdx.x == 0) lse[(int64_t)r * kH + h] = den > 0.f ? mx + logf(den) : -INFINITY;
 }
 
+// Fixed scratch for callers that cannot allocate device memory (see
+// launch_attn_tc_static): the split partials of one call, 64 MiB.
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) float g_attn_scratch[kStaticScratchBytes / sizeof(float)];
+
 }  // namespace
 
 bool attn_tc_supported(int H, int D_K, int D_V) { return H == kH && D_K == kDK && D_V == kDV; }
@@ -561,6 +566,32 @@ dsa_status_t launch_attn_tc(const Rows& R, int32_t row0, int32_t nrows, const ui
     if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   }
   return DSA_OK;
+}
+
+size_t attn_tc_static_scratch_bytes() { return kStaticScratchBytes; }
+
+// Same computation as launch_attn_tc, with the split partials placed in
+// g_attn_scratch instead of a caller workspace.  The array's device address
+// is looked up once per device, with that device current; host code may not
+// use the symbol itself (it names a host-side shadow, not device memory).
+dsa_status_t launch_attn_tc_static(const Rows& R, int32_t row0, int32_t nrows, const uint16_t* q,
+                                   const uint16_t* kv, const int32_t* idx, int k, float sm_scale,
+                                   uint16_t* out, float* lse, cudaStream_t st) {
+  const size_t need = attn_tc_workspace(nrows, k, kH, kDV);
+  if (need > kStaticScratchBytes) return DSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (need) {
+    static void* addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DSA_ERR_CUDA;
+    if (!addr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
+      addr[dev] = p;
+    }
+    scratch = addr[dev];
+  }
+  return launch_attn_tc(R, row0, nrows, q, kv, idx, k, sm_scale, out, lse, scratch, need, st);
 }
 
 }  // namespace dsa

@@ -239,6 +239,27 @@ dsa_status_t dsa_sparse_mla_attn(const dsa_layout_t* layout, const void* q, cons
                   ws_bytes, (cudaStream_t)stream);
 }
 
+dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_layout_t* layout, const void* q,
+                                         const void* kv, const int32_t* idx, int32_t k, int32_t H,
+                                         int32_t D_K, int32_t D_V, float sm_scale, void* out,
+                                         float* lse, void* stream) {
+  Rows R;
+  dsa_status_t s = check_layout(layout, &R);
+  if (s) return s;
+  if ((s = check_attn(R, q, kv, k, H, D_K, D_V, sm_scale, out, lse))) return s;
+  if (!ptr_ok(idx, R.n_q > 0)) return DSA_ERR_INVALID_ARGUMENT;
+  if (attn_tc_supported(H, D_K, D_V) &&
+      attn_tc_workspace(R.n_q, k, H, D_V) > attn_tc_static_scratch_bytes())
+    return DSA_ERR_WORKSPACE;
+  if (R.n_q == 0) return DSA_OK;
+  if ((s = device_rows(&R))) return s;
+  if (attn_tc_supported(H, D_K, D_V))
+    return launch_attn_tc_static(R, 0, R.n_q, (const uint16_t*)q, (const uint16_t*)kv, idx, k,
+                                 sm_scale, (uint16_t*)out, lse, (cudaStream_t)stream);
+  return launch_attn_simt(R, 0, R.n_q, (const uint16_t*)q, (const uint16_t*)kv, idx, k, H, D_K,
+                          D_V, sm_scale, (uint16_t*)out, lse, (cudaStream_t)stream);
+}
+
 size_t dsa_forward_workspace_size(const dsa_layout_t* layout, const dsa_forward_args_t* a) {
   Rows R;
   if (!a || check_layout(layout, &R)) return 0;

@@ -39,4 +39,11 @@ dsa_status_t launch_attn_tc(const Rows& R, int32_t row0, int32_t nrows, const ui
                             const uint16_t* kv, const int32_t* idx, int k, float sm_scale,
                             uint16_t* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st);
 
+// As launch_attn_tc, with the split partials in a fixed static device array
+// (DSA_ERR_WORKSPACE when the call needs more than it holds).
+size_t attn_tc_static_scratch_bytes();
+dsa_status_t launch_attn_tc_static(const Rows& R, int32_t row0, int32_t nrows, const uint16_t* q,
+                                   const uint16_t* kv, const int32_t* idx, int k, float sm_scale,
+                                   uint16_t* out, float* lse, cudaStream_t st);
+
 }  // namespace dsa
