@@ -20,14 +20,18 @@
 // identical softmax decisions).
 //
 // Per CTA: the gathered tile holds the 5 swizzle atoms (64 columns each)
-// 4c .. 4c+4 of 64 selected rows, fetched with TMA tile::gather4 (4 rows per
-// instruction; an empty slot uses an out-of-range row, which reads zeros).
+// 4c .. 4c+4 of 64 selected rows, fetched with 16-byte cp.async by 64
+// producer threads, one row each, written straight into the 128-byte
+// swizzled layout the MMA reads (an empty slot is zero-filled).  Measured on
+// B200: one thread issuing TMA tile::gather4 (4 rows per instruction) needs
+// about 9.3K cycles per such tile, the spread cp.async gather a fraction of it.
 // TMEM: two 64-column score buffers and a 256-column output accumulator.
 //
-// Warp roles (192 threads per CTA):
-//   warp 0     gather producer (indices -> shared memory, TMA gather4)
-//   warp 1     TMEM allocator and MMA issuer (one thread)
-//   warps 2-5  softmax: one thread per head -- score exchange, online softmax
+// Warp roles (352 threads per CTA):
+//   warps 0-1  gather producer (indices -> shared memory, cp.async rows)
+//   warp 2     TMEM allocator and MMA issuer (one thread)
+//   warps 3-10 softmax, two warpgroups: a thread owns one head (its TMEM lane)
+//              and half of each tile's 64 rows -- score exchange, online softmax
 //              in the log2 domain with a lazy rescale (the reference max moves
 //              only when a new score exceeds it by more than 2^8), P to shared
 //              memory as bf16, final normalisation and store.
@@ -46,7 +50,10 @@ namespace {
 
 constexpr int kH = 128, kDK = 576, kDV = 512;
 constexpr int kNT = 64;         // selected rows per tile
-constexpr int kThreads = 192;
+constexpr int kProducers = 64;  // warps 0-1
+constexpr int kSoftmax0 = 96;   // first softmax thread (warps 3-10)
+constexpr int kSoftmaxThreads = 256;
+constexpr int kThreads = kSoftmax0 + kSoftmaxThreads;  // 352
 constexpr int kAtoms = 5;       // 64-column atoms held per CTA
 constexpr int kQBytes = kAtoms * kH * 128;    // 81920
 constexpr int kCBytes = kAtoms * kNT * 128;   // 40960 per stage
@@ -57,8 +64,10 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_C = OFF_Q + kQBytes;
 constexpr int OFF_P = OFF_C + kStages * kCBytes;
 constexpr int OFF_X = OFF_P + 2 * kPBytes;
-constexpr int OFF_IDX = OFF_X + kXBytes;
-constexpr int OFF_BAR = OFF_IDX + kStages * kNT * 4;
+constexpr int OFF_IDX = OFF_X + kXBytes;                 // [stage][64] int32
+constexpr int OFF_MASK = OFF_IDX + kStages * kNT * 4;    // [stage][2] uint32 validity bits
+constexpr int OFF_HMAX = OFF_MASK + kStages * 2 * 4;     // [2 warpgroups][128] float
+constexpr int OFF_BAR = OFF_HMAX + 2 * kH * 4;
 constexpr int kNumBars = 16;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int kSmem = OFF_MISC + 16 + 1024;
@@ -123,14 +132,6 @@ __device__ __forceinline__ bool wait_cluster(uint32_t bar, uint32_t parity, unsi
   }
   return true;
 }
-__device__ __forceinline__ void gather4(uint32_t dst, const CUtensorMap* m, int32_t x, int32_t r0,
-                                        int32_t r1, int32_t r2, int32_t r3, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -144,6 +145,29 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "f"(v[29]), "f"(v[30]), "f"(v[31])
       : "memory");
 }
+// Named barrier `id` over `n` threads, returning the AND of `v` (every
+// participant must reach it, so failures are folded in rather than
+// branched around).
+template <int ID, int N>
+__device__ __forceinline__ bool bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(ID), "n"(N)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&p);
@@ -165,16 +189,17 @@ __host__ __device__ inline Split plan_split(int32_t nrows, int k) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
-                   const __grid_constant__ CUtensorMap cmap, Rows R, int32_t row0,
-                   const int32_t* __restrict__ idx, int k, float scale2, Split sp,
-                   uint16_t* __restrict__ out, float* __restrict__ lse,
+    attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const uint16_t* __restrict__ kv,
+                   Rows R, int32_t row0, const int32_t* __restrict__ idx, int k, float scale2,
+                   Split sp, uint16_t* __restrict__ out, float* __restrict__ lse,
                    float* __restrict__ part_o, float* __restrict__ part_lse) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   int32_t* sidx = reinterpret_cast<int32_t*>(smem + OFF_IDX);
+  uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + OFF_MASK);
+  float* hmax = reinterpret_cast<float*>(smem + OFF_HMAX);
   auto bar = [&](int i) { return sb + OFF_BAR + 8u * i; };
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
@@ -192,20 +217,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(bar(B_QFULL), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(B_CFULL + i), 1);
+      // per producer: a release-arrive after its index store and a cp.async arrive
+      mbar_init(bar(B_CFULL + i), 2 * kProducers);
       mbar_init(bar(B_CEMPTY + i), 1);
       mbar_init(bar(B_SFULL + i), 1);
-      mbar_init(bar(B_SEMPTY + i), 128);
-      mbar_init(bar(B_PFULL + i), 128);
+      mbar_init(bar(B_SEMPTY + i), kSoftmaxThreads);
+      mbar_init(bar(B_PFULL + i), kSoftmaxThreads);
       mbar_init(bar(B_PVDONE + i), 1);
     }
-    mbar_init(bar(B_XFULL), 128);   // the peer's 128 softmax threads
-    mbar_init(bar(B_XEMPTY), 128);
+    mbar_init(bar(B_XFULL), 1);  // one release-arrive from the peer per tile
+    mbar_init(bar(B_XEMPTY), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 2) {
     tmem_alloc(sb + OFF_MISC, 512);
     tmem_relinquish();
   }
@@ -214,60 +240,63 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp < 2) {
     // ------------------------------------------------------------ gather producer
-    if (lane == 0) {
+    if (tid == 0) {
       tma_prefetch(&qmap);
-      tma_prefetch(&cmap);
       mbar_expect_tx(bar(B_QFULL), kQBytes);
       for (int la = 0; la < kAtoms; ++la)
         tma_load_2d(sb + OFF_Q + la * kH * 128, &qmap, (int)(4 * crank + la) * 64, r * kH,
                     bar(B_QFULL));
     }
-    int issued = 0;
+    const uint16_t* kvb = kv + ri.kbase * kDK + 256 * crank;  // atoms 4c .. 4c+4
+    auto load_idx = [&](int n) -> int32_t {
+      const int slot = slot_lo + n * kNT + tid;
+      int32_t s = slot < slot_hi ? __ldg(idx + (int64_t)rloc * k + slot) : -1;
+      if (s < -1 || s >= ri.len || ri.t < 0) {
+        if (s != -1 && ri.t >= 0) raise_status(R, kErrBadIndex);
+        s = -1;
+      }
+      return s;
+    };
+    // A warp instruction copies 4 rows x 128 contiguous bytes: lanes 8g..8g+7
+    // take the 16-byte chunks of row 4j+g of this warp's 32 rows.
+    const int sub = lane >> 3, ch = lane & 7;
+    int32_t pre = ntiles > 0 ? load_idx(0) : -1;
     for (int n = 0; n < ntiles; ++n) {
       const int st = n & 1;
-      if (!mbar_wait(bar(B_CEMPTY + st), ((n >> 1) & 1) ^ 1, R.status) || *abort_flag) {
+      const bool ok = mbar_wait(bar(B_CEMPTY + st), ((n >> 1) & 1) ^ 1, R.status) && !*abort_flag;
+      if (!bar_and<2, kProducers>(ok)) {
         *abort_flag = 1;
         break;
       }
-      int32_t* si = sidx + st * kNT;
-      for (int j = lane; j < kNT; j += 32) {
-        const int slot = slot_lo + n * kNT + j;
-        int32_t s = slot < slot_hi ? __ldg(idx + (int64_t)rloc * k + slot) : -1;
-        if (s < -1 || s >= ri.len || ri.t < 0) {
-          if (s != -1 && ri.t >= 0) raise_status(R, kErrBadIndex);
-          s = -1;
-        }
-        si[j] = s;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_expect_tx(bar(B_CFULL + st), kCBytes);
-        const int64_t kb = ri.kbase;
-        for (int la = 0; la < kAtoms; ++la) {
-          const int x = (int)(4 * crank + la) * 64;
-          for (int g = 0; g < kNT / 4; ++g) {
-            int32_t rr[4];
+      sidx[st * kNT + tid] = pre;
+      const uint32_t bits = __ballot_sync(0xffffffffu, pre >= 0);
+      if (lane == 0) vmask[st * 2 + warp] = bits;
+      mbar_arrive(bar(B_CFULL + st));  // publishes indices and mask to the softmax threads
+      asm volatile("bar.sync 2, 64;" ::: "memory");  // every producer sees the tile's indices
+      pre = n + 1 < ntiles ? load_idx(n + 1) : -1;    // overlaps the copies below
+      const uint32_t cb = sb + OFF_C + st * kCBytes;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int32_t s = si[4 * g + i];
-              rr[i] = s >= 0 ? (int32_t)(kb + s) : -1;  // -1: out of range, reads zeros
-            }
-            gather4(sb + OFF_C + st * kCBytes + la * kNT * 128 + g * 512, &cmap, x, rr[0], rr[1],
-                    rr[2], rr[3], bar(B_CFULL + st));
-          }
-        }
+      for (int j = 0; j < 8; ++j) {
+        const int row = warp * 32 + 4 * j + sub;
+        const int32_t s = sidx[st * kNT + row];
+        const char* src = reinterpret_cast<const char*>(s >= 0 ? kvb + (int64_t)s * kDK : kv);
+        const uint32_t nbytes = s >= 0 ? 16u : 0u;  // 0: zero-fill
+        const uint32_t dst = cb + row * 128 + ((uint32_t)(ch ^ (row & 7)) << 4);
+#pragma unroll
+        for (int la = 0; la < kAtoms; ++la)
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst + la * kNT * 128),
+                       "l"(src + (la * 64 + ch * 8) * 2), "r"(nbytes)
+                       : "memory");
       }
-      __syncwarp();
-      ++issued;
+      // arrives on the stage barrier once this thread's copies have landed
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_CFULL + st))
+                   : "memory");
     }
-    if (lane == 0) {  // leave no copy in flight behind us
-      for (int n = max(0, issued - kStages); n < issued; ++n)
-        mbar_wait(bar(B_CFULL + (n & 1)), (n >> 1) & 1, R.status);
-      mbar_wait(bar(B_QFULL), 0, R.status);
-    }
-  } else if (warp == 1) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (tid == 0) mbar_wait(bar(B_QFULL), 0, R.status);
+  } else if (warp == 2) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(bar(B_QFULL), 0, R.status);
@@ -280,11 +309,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // cp.async rows
           tc_fence_after();
           const uint32_t cb = sb + OFF_C + st * kCBytes;
 #pragma unroll
           for (int kk = 0; kk < 18; ++kk) {
-            const int e = 288 * (int)crank + 16 * kk;       // global contraction index
+            const int e = 288 * (int)crank + 16 * kk;  // global contraction index
             const int la = e / 64 - 4 * (int)crank, off = (e % 64) * 2;
             mma_bf16(tmem + TM_S + st * kNT, desc_sw128(qb + la * kH * 128 + off, 1024),
                      desc_sw128(cb + la * kNT * 128 + off, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
@@ -317,6 +347,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
+    // Two warpgroups; warpgroup wg handles tokens 32wg .. 32wg+31 of every
+    // tile for the head of its TMEM lane.
+    const int wg = (warp - 3) >> 2;
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -326,110 +359,120 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t xempty_peer = map_peer(bar(B_XEMPTY), peer);
     float m2 = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int n = 0; n < ntiles && ok; ++n) {
+    for (int n = 0; n < ntiles; ++n) {
       const int st = n & 1;
-      bool w_ok = mbar_wait(bar(B_CFULL + st), (n >> 1) & 1, R.status) &&
-                  mbar_wait(bar(B_SFULL + st), (n >> 1) & 1, R.status) && !*abort_flag;
-      if (!__all_sync(0xffffffffu, w_ok)) {  // warp-uniform: TMEM loads are warp-collective
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float s[kNT];
-      {
-        float a[32], b[32];
-        tmem_ld32(tmem + lane_off + TM_S + st * kNT, a);
-        tmem_ld32(tmem + lane_off + TM_S + st * kNT + 32, b);
+      bool w_ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CFULL + st), (n >> 1) & 1, R.status) &&
+                                              mbar_wait(bar(B_SFULL + st), (n >> 1) & 1, R.status) &&
+                                              !*abort_flag);
+      float s[32];
+      if (w_ok) {
+        tc_fence_after();
+        tmem_ld32(tmem + lane_off + TM_S + st * kNT + 32 * wg, s);
+        tc_fence_before();
+      } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          s[j] = a[j];
-          s[32 + j] = b[j];
+        for (int j = 0; j < 32; ++j) s[j] = 0.f;
+      }
+      mbar_arrive(bar(B_SEMPTY + st));
+      // send this half of the partial scores to the peer CTA
+      w_ok = w_ok && __all_sync(0xffffffffu, mbar_wait(bar(B_XEMPTY), (n & 1) ^ 1, R.status));
+      if (w_ok) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int cc = 8 * wg + c;
+          st_cluster_v4(xrow_peer + ((cc ^ (h & 7)) * 16), s[4 * c], s[4 * c + 1], s[4 * c + 2],
+                        s[4 * c + 3]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(B_SEMPTY + st));
-      // exchange the partial scores with the peer CTA
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_XEMPTY), (n & 1) ^ 1, R.status))) {
+      if (!bar_and<1, kSoftmaxThreads>(w_ok)) {  // all stores issued: one cumulative release
         ok = false;
         break;
       }
+      if (tid == kSoftmax0) arrive_remote(xfull_peer);
+      w_ok = __all_sync(0xffffffffu, wait_cluster(bar(B_XFULL), n & 1, R.status));
+      const uint32_t bits = vmask[st * 2 + wg];
+      float hm = -INFINITY;
+      {
+        const float4* xr = reinterpret_cast<const float4*>(smem + OFF_X + h * (kNT * 4));
 #pragma unroll
-      for (int c = 0; c < kNT / 4; ++c)
-        st_cluster_v4(xrow_peer + ((c ^ (h & 7)) * 16), s[4 * c], s[4 * c + 1], s[4 * c + 2],
-                      s[4 * c + 3]);
-      arrive_remote(xfull_peer);
-      if (!__all_sync(0xffffffffu, wait_cluster(bar(B_XFULL), n & 1, R.status))) {
+        for (int c = 0; c < 8; ++c) {
+          const int cc = 8 * wg + c;
+          const float4 v = w_ok ? xr[cc ^ (h & 7)] : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * c + e;
+            s[j] = ((bits >> j) & 1u) ? (s[j] + vv[e]) * scale2 : -INFINITY;
+            hm = fmaxf(hm, s[j]);
+          }
+        }
+      }
+      hmax[wg * kH + h] = hm;
+      if (!bar_and<1, kSoftmaxThreads>(w_ok)) {  // exchange buffer read, half maxima visible
         ok = false;
         break;
       }
-      const float4* xr = reinterpret_cast<const float4*>(smem + OFF_X + h * (kNT * 4));
-#pragma unroll
-      for (int c = 0; c < kNT / 4; ++c) {
-        const float4 v = xr[c ^ (h & 7)];
-        s[4 * c] += v.x;
-        s[4 * c + 1] += v.y;
-        s[4 * c + 2] += v.z;
-        s[4 * c + 3] += v.w;
-      }
-      arrive_remote(xempty_peer);
-      // online softmax in the log2 domain
-      const int32_t* si = sidx + st * kNT;
-      float mt = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < kNT; ++j) {
-        s[j] = si[j] >= 0 ? s[j] * scale2 : -INFINITY;
-        mt = fmaxf(mt, s[j]);
-      }
+      if (tid == kSoftmax0) arrive_remote(xempty_peer);
+      const float mt = fmaxf(hm, hmax[(wg ^ 1) * kH + h]);  // same value in both warpgroups
+      bool t_ok = true;
       if (mt > m2 + kRescale || (m2 == -INFINITY && mt != -INFINITY)) {
         const float m_new = fmaxf(mt, m2);
-        const float alpha = exp2f(m2 - m_new);  // 0 when m2 = -inf
+        const float alpha = ex2(m2 - m_new);  // 0 when m2 = -inf
         l *= alpha;
-        if (n > 0) {  // rescale the output accumulated so far (PV of tile n-1 first)
+        if (n > 0) {  // rescale this warpgroup's 128 output columns (PV of tile n-1 first)
           const int m = n - 1;
-          if (!__all_sync(0xffffffffu,
-                          mbar_wait(bar(B_PVDONE + (m & 1)), (m >> 1) & 1, R.status))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          for (int cc = 0; cc < 8; ++cc) {
-            float v[32];
-            tmem_ld32(tmem + lane_off + TM_O + cc * 32, v);
+          t_ok = __all_sync(0xffffffffu,
+                            mbar_wait(bar(B_PVDONE + (m & 1)), (m >> 1) & 1, R.status));
+          if (t_ok) {
+            tc_fence_after();
+            for (int cc = 0; cc < 4; ++cc) {
+              float v[32];
+              const uint32_t ta = tmem + lane_off + TM_O + 128 * wg + cc * 32;
+              tmem_ld32(ta, v);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= alpha;
-            tmem_st32(tmem + lane_off + TM_O + cc * 32, v);
+              for (int j = 0; j < 32; ++j) v[j] *= alpha;
+              tmem_st32(ta, v);
+            }
           }
         }
         m2 = m_new;
       }
       // P buffer n&1 is free once PV(n-2) completed
-      if (n >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE + (n & 1)), ((n - 2) >> 1) & 1, R.status))) {
-        ok = false;
-        break;
-      }
+      if (n >= 2)
+        t_ok = t_ok && __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE + (n & 1)),
+                                                         ((n - 2) >> 1) & 1, R.status));
       uint8_t* prow = smem + OFF_P + (n & 1) * kPBytes + h * 128;
       const float mref = m2 == -INFINITY ? 0.f : m2;  // all scores -inf: p = 0
       float lsum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint32_t w4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float p0 = exp2f(s[8 * c + 2 * e] - mref);
-          const float p1 = exp2f(s[8 * c + 2 * e + 1] - mref);
+          const float p0 = ex2(s[8 * c + 2 * e] - mref);
+          const float p1 = ex2(s[8 * c + 2 * e + 1] - mref);
           w4[e] = pack_bf16(p0, p1);  // bf16 only as the MMA operand
           lsum += p0 + p1;            // the denominator keeps fp32 probabilities
         }
-        *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        const int cc = 4 * wg + c;
+        if (t_ok)
+          *reinterpret_cast<uint4*>(prow + ((cc ^ (h & 7)) * 16)) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
       l += lsum;
+      if (!t_ok) *abort_flag = 1;  // seen by everyone at the next barrier reduction
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P: generic -> async proxy
       tc_fence_before();  // orders a rescale's tcgen05.st before the next MMA
       mbar_arrive(bar(B_PFULL + (n & 1)));
     }
     if (!ok) *abort_flag = 1;
-    // final output
+    // combine the two warpgroups' denominators (the first barrier retires the
+    // last tile's reads of the half maxima)
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    hmax[wg * kH + h] = l;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    l += hmax[(wg ^ 1) * kH + h];
+    // final output: warpgroup wg writes columns 128wg .. 128wg+127 of this CTA's half
     bool have_o = ok && ntiles > 0;
     if (have_o) {
       const int m = ntiles - 1;
@@ -440,15 +483,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const float inv = l > 0.f ? 1.f / l : 0.f;
     const float lse_v = l > 0.f ? (m2 + log2f(l)) * kLn2 : -INFINITY;
     const bool final_out = sp.nsplit == 1;
-    for (int cc = 0; cc < 8; ++cc) {
+    for (int cc = 0; cc < 4; ++cc) {
       float v[32];
+      const int c32 = 4 * wg + cc;  // 32-column block inside this CTA's 256 columns
       if (have_o) {
-        tmem_ld32(tmem + lane_off + TM_O + cc * 32, v);
+        tmem_ld32(tmem + lane_off + TM_O + c32 * 32, v);
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = 0.f;
       }
-      const int col = (int)crank * 256 + cc * 32;
+      const int col = (int)crank * 256 + c32 * 32;
       if (final_out) {
         uint16_t* o = out + ((int64_t)r * kH + h) * kDV + col;
 #pragma unroll
@@ -466,7 +510,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                          v[4 * q4 + 2] * inv, v[4 * q4 + 3] * inv);
       }
     }
-    if (crank == 0) {
+    if (crank == 0 && wg == 0) {
       if (final_out) {
         if (lse) lse[(int64_t)r * kH + h] = lse_v;
       } else {
@@ -477,7 +521,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -548,16 +592,15 @@ dsa_status_t launch_attn_tc(const Rows& R, int32_t row0, int32_t nrows, const ui
     part_o = reinterpret_cast<float*>(ws);
     part_lse = part_o + (size_t)nrows * sp.nsplit * kH * kDV;
   }
-  CUtensorMap qmap, cmap;
+  CUtensorMap qmap;
   if (!make_tmap_2d(&qmap, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, (uint64_t)R.n_q * kH, 64,
-                    kH) ||
-      !make_tmap_2d(&cmap, kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, (uint64_t)R.n_k, 64, 1))
+                    kH))
     return DSA_ERR_CUDA;
   if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
   const dim3 grid(2 * nrows * sp.nsplit);
-  attn_tc_kernel<<<grid, kThreads, kSmem, st>>>(qmap, cmap, R, row0, idx, k, sm_scale * kLog2e,
+  attn_tc_kernel<<<grid, kThreads, kSmem, st>>>(qmap, kv, R, row0, idx, k, sm_scale * kLog2e,
                                                 sp, out, lse, part_o, part_lse);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (sp.nsplit > 1) {
