@@ -22,19 +22,29 @@
 // Per CTA: the gathered tile holds the 5 swizzle atoms (64 columns each)
 // 4c .. 4c+4 of 64 selected rows, fetched with 16-byte cp.async by 64
 // producer threads, one row each, written straight into the 128-byte
-// swizzled layout the MMA reads (an empty slot is zero-filled).  Measured on
-// B200: one thread issuing TMA tile::gather4 (4 rows per instruction) needs
-// about 9.3K cycles per such tile, the spread cp.async gather a fraction of it.
-// TMEM: two 64-column score buffers and a 256-column output accumulator.
+// swizzled layout the MMA reads (an empty slot is zero-filled); 4 such
+// stages are in flight.  Measured on B200: one thread issuing TMA
+// tile::gather4 (4 rows per instruction) needs about 9.3K cycles per such
+// tile, the spread cp.async gather a fraction of it.
+//
+// Both products take their A operand from TMEM (the .ts form), so shared
+// memory holds only gathered rows and the exchange buffers:
+//   columns   0..143  the CTA's 288 query dims of every head, bf16 pairs
+//   columns 160..223  the 64-column partial score tile (fp32)
+//   columns 224..255  P, the tile's probabilities as bf16 pairs
+//   columns 256..511  the 256-column output accumulator
 //
 // Warp roles (352 threads per CTA):
 //   warps 0-1  gather producer (indices -> shared memory, cp.async rows)
-//   warp 2     TMEM allocator and MMA issuer (one thread)
+//   warp 2     TMEM allocator and MMA issuer (one thread, issues whichever of
+//              QK(next tile) and PV(oldest tile with P ready) can go)
 //   warps 3-10 softmax, two warpgroups: a thread owns one head (its TMEM lane)
-//              and half of each tile's 64 rows -- score exchange, online softmax
-//              in the log2 domain with a lazy rescale (the reference max moves
-//              only when a new score exceeds it by more than 2^8), P to shared
-//              memory as bf16, final normalisation and store.
+//              and half of each tile's 64 rows.  Software-pipelined: tile
+//              n+1's partial scores leave for the peer before tile n's
+//              softmax runs (double-buffered exchange).  Online softmax in
+//              the log2 domain with a lazy rescale (the reference max moves
+//              only when a new score exceeds it by more than 2^8), P to TMEM
+//              as bf16, final normalisation and store.
 // Decode rows are split over several clusters; each writes a normalised
 // partial output and its log-sum-exp, merged by attn_combine_kernel.
 #include <cudaTypedefs.h>
@@ -55,25 +65,25 @@ constexpr int kSoftmax0 = 96;   // first softmax thread (warps 3-10)
 constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmax0 + kSoftmaxThreads;  // 352
 constexpr int kAtoms = 5;       // 64-column atoms held per CTA
-constexpr int kQBytes = kAtoms * kH * 128;    // 81920
 constexpr int kCBytes = kAtoms * kNT * 128;   // 40960 per stage
-constexpr int kStages = 2;
-constexpr int kPBytes = kH * kNT * 2;         // 16384 per buffer
-constexpr int kXBytes = kH * kNT * 4;         // 32768
-constexpr int OFF_Q = 0;
-constexpr int OFF_C = OFF_Q + kQBytes;
-constexpr int OFF_P = OFF_C + kStages * kCBytes;
-constexpr int OFF_X = OFF_P + 2 * kPBytes;
-constexpr int OFF_IDX = OFF_X + kXBytes;                 // [stage][64] int32
+constexpr int kStages = 4;
+constexpr int kXBytes = kH * kNT * 4;         // 32768 per exchange buffer
+constexpr int OFF_C = 0;
+constexpr int OFF_X = OFF_C + kStages * kCBytes;         // [2] exchange buffers
+constexpr int OFF_IDX = OFF_X + 2 * kXBytes;             // [stage][64] int32
 constexpr int OFF_MASK = OFF_IDX + kStages * kNT * 4;    // [stage][2] uint32 validity bits
 constexpr int OFF_HMAX = OFF_MASK + kStages * 2 * 4;     // [2 warpgroups][128] float
 constexpr int OFF_BAR = OFF_HMAX + 2 * kH * 4;
-constexpr int kNumBars = 16;
+constexpr int kNumBars = 20;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
-constexpr int kSmem = OFF_MISC + 16 + 1024;
+// The dynamic window starts 1024-aligned (right after the driver's reserved
+// kilobyte, with no static shared memory); the kernel checks it.
+constexpr int kSmem = OFF_MISC + 16;
 static_assert(kSmem <= 232448, "shared memory");
 // TMEM columns
-constexpr uint32_t TM_S = 0;     // two 64-column score buffers
+constexpr uint32_t TM_Q = 0;     // the CTA's 288 query dims of all heads, bf16 pairs (144 cols)
+constexpr uint32_t TM_S = 160;   // 64-column score tile
+constexpr uint32_t TM_P = 224;   // 32-column bf16 P tile (the PV A operand)
 constexpr uint32_t TM_O = 256;   // 256-column output accumulator
 constexpr uint32_t IDESC_QK = idesc(1, 128, kNT);
 constexpr uint32_t IDESC_PV = idesc(1, 128, 256, false, true);
@@ -82,8 +92,16 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;  // log2 headroom before the reference max moves
 
 enum {
-  B_QFULL = 0, B_CFULL = 1, B_CEMPTY = 3, B_SFULL = 5, B_SEMPTY = 7, B_PFULL = 9,
-  B_PVDONE = 11, B_XFULL = 13, B_XEMPTY = 14, B_DRAIN = 15
+  B_QREADY = 0,  // the query is in TMEM (every softmax thread)
+  B_CFULL = 1,   // [4] stage rows landed (producers)
+  B_CEMPTY = 5,  // [4] PV of the stage retired
+  B_SFULL = 9,   // QK retired
+  B_SEMPTY = 10, // scores read (every softmax thread)
+  B_PFULL = 11,  // P stored in TMEM (every softmax thread)
+  B_PVDONE = 12, // PV retired
+  B_XFULL = 13,  // [2] the peer's partial scores arrived
+  B_XEMPTY = 15, // [2] the peer read our partial scores
+  B_DRAIN = 17
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -145,6 +163,34 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "f"(v[29]), "f"(v[30]), "f"(v[31])
       : "memory");
 }
+// MMA with the A operand in TMEM (rows in lanes, 16-bit K pairs per column).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                            uint32_t id, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(id), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
 // Named barrier `id` over `n` threads, returning the AND of `v` (every
 // participant must reach it, so failures are folded in rather than
 // branched around).
@@ -189,14 +235,17 @@ __host__ __device__ inline Split plan_split(int32_t nrows, int k) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const uint16_t* __restrict__ kv,
-                   Rows R, int32_t row0, const int32_t* __restrict__ idx, int k, float scale2,
-                   Split sp, uint16_t* __restrict__ out, float* __restrict__ lse,
+    attn_tc_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kv, Rows R,
+                   int32_t row0, const int32_t* __restrict__ idx, int k, float scale2, Split sp,
+                   uint16_t* __restrict__ out, float* __restrict__ lse,
                    float* __restrict__ part_o, float* __restrict__ part_lse) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t sb = smem_u32(smem);
+  if (sb & 1023u) {  // the swizzled operand layouts need 1024-byte alignment
+    if (threadIdx.x == 0) raise_status(R, kErrLayout);
+    return;  // uniform across the cluster: both CTAs share the layout
+  }
   int32_t* sidx = reinterpret_cast<int32_t*>(smem + OFF_IDX);
   uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + OFF_MASK);
   float* hmax = reinterpret_cast<float*>(smem + OFF_HMAX);
@@ -215,18 +264,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int ntiles = slot_hi > slot_lo ? (slot_hi - slot_lo + kNT - 1) / kNT : 0;
 
   if (tid == 0) {
-    mbar_init(bar(B_QFULL), 1);
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(bar(B_QREADY), kSoftmaxThreads);
+    for (int i = 0; i < kStages; ++i) {
       // per producer: a release-arrive after its index store and a cp.async arrive
       mbar_init(bar(B_CFULL + i), 2 * kProducers);
       mbar_init(bar(B_CEMPTY + i), 1);
-      mbar_init(bar(B_SFULL + i), 1);
-      mbar_init(bar(B_SEMPTY + i), kSoftmaxThreads);
-      mbar_init(bar(B_PFULL + i), kSoftmaxThreads);
-      mbar_init(bar(B_PVDONE + i), 1);
     }
-    mbar_init(bar(B_XFULL), 1);  // one release-arrive from the peer per tile
-    mbar_init(bar(B_XEMPTY), 1);
+    mbar_init(bar(B_SFULL), 1);
+    mbar_init(bar(B_SEMPTY), kSoftmaxThreads);
+    mbar_init(bar(B_PFULL), kSoftmaxThreads);
+    mbar_init(bar(B_PVDONE), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_XFULL + i), 1);  // one release-arrive from the peer per tile
+      mbar_init(bar(B_XEMPTY + i), 1);
+    }
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -242,13 +293,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp < 2) {
     // ------------------------------------------------------------ gather producer
-    if (tid == 0) {
-      tma_prefetch(&qmap);
-      mbar_expect_tx(bar(B_QFULL), kQBytes);
-      for (int la = 0; la < kAtoms; ++la)
-        tma_load_2d(sb + OFF_Q + la * kH * 128, &qmap, (int)(4 * crank + la) * 64, r * kH,
-                    bar(B_QFULL));
-    }
     const uint16_t* kvb = kv + ri.kbase * kDK + 256 * crank;  // atoms 4c .. 4c+4
     auto load_idx = [&](int n) -> int32_t {
       const int slot = slot_lo + n * kNT + tid;
@@ -264,8 +308,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int sub = lane >> 3, ch = lane & 7;
     int32_t pre = ntiles > 0 ? load_idx(0) : -1;
     for (int n = 0; n < ntiles; ++n) {
-      const int st = n & 1;
-      const bool ok = mbar_wait(bar(B_CEMPTY + st), ((n >> 1) & 1) ^ 1, R.status) && !*abort_flag;
+      const int st = n % kStages;
+      const bool ok = mbar_wait(bar(B_CEMPTY + st), ((n / kStages) & 1) ^ 1, R.status) &&
+                      !*abort_flag;
       if (!bar_and<2, kProducers>(ok)) {
         *abort_flag = 1;
         break;
@@ -295,48 +340,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                    : "memory");
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-    if (tid == 0) mbar_wait(bar(B_QFULL), 0, R.status);
   } else if (warp == 2) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait(bar(B_QFULL), 0, R.status);
-      const uint32_t qb = sb + OFF_Q;
-      for (int n = 0; ok && n <= ntiles; ++n) {
-        if (n < ntiles) {
-          const int st = n & 1;
-          if (!mbar_wait(bar(B_CFULL + st), (n >> 1) & 1, R.status) ||
-              !mbar_wait(bar(B_SEMPTY + st), ((n >> 1) & 1) ^ 1, R.status) || *abort_flag) {
-            ok = false;
-            break;
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // cp.async rows
-          tc_fence_after();
-          const uint32_t cb = sb + OFF_C + st * kCBytes;
-#pragma unroll
-          for (int kk = 0; kk < 18; ++kk) {
-            const int e = 288 * (int)crank + 16 * kk;  // global contraction index
-            const int la = e / 64 - 4 * (int)crank, off = (e % 64) * 2;
-            mma_bf16(tmem + TM_S + st * kNT, desc_sw128(qb + la * kH * 128 + off, 1024),
-                     desc_sw128(cb + la * kNT * 128 + off, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar(B_SFULL + st));
+      bool ok = mbar_wait(bar(B_QREADY), 0, R.status);
+      // Issue whichever is ready: QK of the next tile (rows landed, score
+      // tile free) or PV of the oldest tile whose P is in TMEM.  PV never
+      // waits for a later tile's rows.
+      int nq = 0, np = 0;
+      long long t0 = clock64();
+      while (ok && np < ntiles) {
+        if (*abort_flag) {
+          ok = false;
+          break;
         }
-        if (n >= 1) {
-          const int m = n - 1, pb = m & 1;
-          if (!mbar_wait(bar(B_PFULL + pb), (m >> 1) & 1, R.status) || *abort_flag) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t cb = sb + OFF_C + pb * kCBytes;  // stage of tile m
-          const uint32_t pbase = sb + OFF_P + pb * kPBytes;
+        bool progressed = false;
+        if (nq < ntiles) {
+          const int st = nq % kStages;
+          if (mbar_try(bar(B_CFULL + st), (nq / kStages) & 1) &&
+              mbar_try(bar(B_SEMPTY), (nq & 1) ^ 1)) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // cp.async rows
+            tc_fence_after();
+            const uint32_t cb = sb + OFF_C + st * kCBytes;
 #pragma unroll
-          for (int kk = 0; kk < kNT / 16; ++kk)
-            mma_bf16(tmem + TM_O, desc_sw128(pbase + kk * 32, 1024),
-                     desc_sw128_mn(cb + kk * 2048, kNT * 128, 1024), IDESC_PV,
-                     (m > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar(B_PVDONE + pb));
-          mma_commit(bar(B_CEMPTY + pb));
+            for (int kk = 0; kk < 18; ++kk) {
+              const int e = 288 * (int)crank + 16 * kk;  // global contraction index
+              const int la = e / 64 - 4 * (int)crank, off = (e % 64) * 2;
+              mma_bf16_ts(tmem + TM_S, tmem + TM_Q + 8 * kk,
+                          desc_sw128(cb + la * kNT * 128 + off, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(B_SFULL));
+            ++nq;
+            progressed = true;
+          }
+        }
+        if (np < nq) {
+          if (mbar_try(bar(B_PFULL), np & 1)) {
+            tc_fence_after();
+            const uint32_t cb = sb + OFF_C + (np % kStages) * kCBytes;  // stage of tile np
+#pragma unroll
+            for (int kk = 0; kk < kNT / 16; ++kk)
+              mma_bf16_ts(tmem + TM_O, tmem + TM_P + kk * 8,
+                          desc_sw128_mn(cb + kk * 2048, kNT * 128, 1024), IDESC_PV,
+                          (np > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bar(B_PVDONE));
+            mma_commit(bar(B_CEMPTY + np % kStages));
+            ++np;
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t0 = clock64();
+        } else if (clock64() - t0 > kSpinLimit) {
+          atomicOr(R.status, kErrTimeout);
+          ok = false;
         }
       }
       if (!ok) {
@@ -347,53 +404,95 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    // Two warpgroups; warpgroup wg handles tokens 32wg .. 32wg+31 of every
-    // tile for the head of its TMEM lane.
+    // Two warpgroups; warpgroup wg handles rows 32wg .. 32wg+31 of every
+    // tile for the head of its TMEM lane.  Software-pipelined: the partial
+    // scores of tile n+1 go to the peer before tile n's softmax runs, so the
+    // exchange overlaps the arithmetic (double-buffered exchange buffers).
     const int wg = (warp - 3) >> 2;
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t xrow = sb + OFF_X + h * (kNT * 4);
-    const uint32_t xrow_peer = map_peer(xrow, peer);
-    const uint32_t xfull_peer = map_peer(bar(B_XFULL), peer);
-    const uint32_t xempty_peer = map_peer(bar(B_XEMPTY), peer);
+    // The query: this CTA's 288 contraction dims of head h, as bf16 pairs in
+    // TMEM columns TM_Q .. TM_Q+143 (warpgroup wg stores 72 of them).
+    {
+      const uint4* qsrc = reinterpret_cast<const uint4*>(
+          q + ((int64_t)r * kH + h) * kDK + 288 * crank + 144 * wg);
+#pragma unroll
+      for (int part = 0; part < 3; ++part) {  // 3 x 48 dims = 3 x 24 columns
+        uint32_t w24[24];
+#pragma unroll
+        for (int v = 0; v < 6; ++v) {
+          const uint4 x = __ldg(qsrc + part * 6 + v);
+          w24[4 * v] = x.x;
+          w24[4 * v + 1] = x.y;
+          w24[4 * v + 2] = x.z;
+          w24[4 * v + 3] = x.w;
+        }
+        const uint32_t ta = tmem + lane_off + TM_Q + 72 * wg + 24 * part;
+        uint32_t a8[8], b8[8], c8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          a8[e] = w24[e];
+          b8[e] = w24[8 + e];
+          c8[e] = w24[16 + e];
+        }
+        tmem_st8(ta, a8);
+        tmem_st8(ta + 8, b8);
+        tmem_st8(ta + 16, c8);
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_QREADY));
+    }
+    const uint32_t xrow_peer0 = map_peer(sb + OFF_X + h * (kNT * 4), peer);
+    const uint32_t xfull_peer0 = map_peer(bar(B_XFULL), peer);
+    const uint32_t xempty_peer0 = map_peer(bar(B_XEMPTY), peer);
     float m2 = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int n = 0; n < ntiles; ++n) {
-      const int st = n & 1;
-      bool w_ok = __all_sync(0xffffffffu, mbar_wait(bar(B_CFULL + st), (n >> 1) & 1, R.status) &&
-                                              mbar_wait(bar(B_SFULL + st), (n >> 1) & 1, R.status) &&
-                                              !*abort_flag);
-      float s[32];
+    float s_cur[32], s_nxt[32];
+    // Loads tile m's partial scores into d and ships them to the peer.
+    auto send = [&](int m, float (&d)[32]) -> bool {
+      const int st = m % kStages, xb = m & 1;
+      bool w_ok = __all_sync(0xffffffffu,
+                             mbar_wait(bar(B_CFULL + st), (m / kStages) & 1, R.status) &&
+                                 mbar_wait(bar(B_SFULL), m & 1, R.status) && !*abort_flag);
       if (w_ok) {
         tc_fence_after();
-        tmem_ld32(tmem + lane_off + TM_S + st * kNT + 32 * wg, s);
+        tmem_ld32(tmem + lane_off + TM_S + 32 * wg, d);
         tc_fence_before();
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) s[j] = 0.f;
+        for (int j = 0; j < 32; ++j) d[j] = 0.f;
       }
-      mbar_arrive(bar(B_SEMPTY + st));
-      // send this half of the partial scores to the peer CTA
-      w_ok = w_ok && __all_sync(0xffffffffu, mbar_wait(bar(B_XEMPTY), (n & 1) ^ 1, R.status));
+      mbar_arrive(bar(B_SEMPTY));
+      w_ok = w_ok && __all_sync(0xffffffffu, mbar_wait(bar(B_XEMPTY + xb), ((m >> 1) & 1) ^ 1,
+                                                       R.status));
       if (w_ok) {
+        const uint32_t xr = xrow_peer0 + xb * kXBytes;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const int cc = 8 * wg + c;
-          st_cluster_v4(xrow_peer + ((cc ^ (h & 7)) * 16), s[4 * c], s[4 * c + 1], s[4 * c + 2],
-                        s[4 * c + 3]);
+          st_cluster_v4(xr + ((cc ^ (h & 7)) * 16), d[4 * c], d[4 * c + 1], d[4 * c + 2],
+                        d[4 * c + 3]);
         }
       }
-      if (!bar_and<1, kSoftmaxThreads>(w_ok)) {  // all stores issued: one cumulative release
+      if (!bar_and<1, kSoftmaxThreads>(w_ok)) return false;  // all stores issued
+      if (tid == kSoftmax0) arrive_remote(xfull_peer0 + 8u * xb);  // one cumulative release
+      return true;
+    };
+    if (ntiles > 0) ok = send(0, s_cur);
+    for (int n = 0; ok && n < ntiles; ++n) {
+      const int st = n % kStages, xb = n & 1;
+      if (n + 1 < ntiles && !send(n + 1, s_nxt)) {
         ok = false;
         break;
       }
-      if (tid == kSoftmax0) arrive_remote(xfull_peer);
-      w_ok = __all_sync(0xffffffffu, wait_cluster(bar(B_XFULL), n & 1, R.status));
+      // the peer's half of tile n
+      bool w_ok = __all_sync(0xffffffffu, wait_cluster(bar(B_XFULL + xb), (n >> 1) & 1, R.status));
       const uint32_t bits = vmask[st * 2 + wg];
       float hm = -INFINITY;
       {
-        const float4* xr = reinterpret_cast<const float4*>(smem + OFF_X + h * (kNT * 4));
+        const float4* xr = reinterpret_cast<const float4*>(smem + OFF_X + xb * kXBytes +
+                                                            h * (kNT * 4));
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const int cc = 8 * wg + c;
@@ -402,8 +501,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int j = 4 * c + e;
-            s[j] = ((bits >> j) & 1u) ? (s[j] + vv[e]) * scale2 : -INFINITY;
-            hm = fmaxf(hm, s[j]);
+            s_cur[j] = ((bits >> j) & 1u) ? (s_cur[j] + vv[e]) * scale2 : -INFINITY;
+            hm = fmaxf(hm, s_cur[j]);
           }
         }
       }
@@ -412,58 +511,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
-      if (tid == kSoftmax0) arrive_remote(xempty_peer);
+      if (tid == kSoftmax0) arrive_remote(xempty_peer0 + 8u * xb);
       const float mt = fmaxf(hm, hmax[(wg ^ 1) * kH + h]);  // same value in both warpgroups
-      bool t_ok = true;
+      // P of tile n-1 is consumed and O is final up to tile n-1 once PV(n-1) retired
+      bool t_ok = n == 0 || __all_sync(0xffffffffu,
+                                       mbar_wait(bar(B_PVDONE), (n - 1) & 1, R.status));
       if (mt > m2 + kRescale || (m2 == -INFINITY && mt != -INFINITY)) {
         const float m_new = fmaxf(mt, m2);
         const float alpha = ex2(m2 - m_new);  // 0 when m2 = -inf
         l *= alpha;
-        if (n > 0) {  // rescale this warpgroup's 128 output columns (PV of tile n-1 first)
-          const int m = n - 1;
-          t_ok = __all_sync(0xffffffffu,
-                            mbar_wait(bar(B_PVDONE + (m & 1)), (m >> 1) & 1, R.status));
-          if (t_ok) {
-            tc_fence_after();
-            for (int cc = 0; cc < 4; ++cc) {
-              float v[32];
-              const uint32_t ta = tmem + lane_off + TM_O + 128 * wg + cc * 32;
-              tmem_ld32(ta, v);
+        if (n > 0 && t_ok) {  // rescale this warpgroup's 128 output columns
+          tc_fence_after();
+          for (int cc = 0; cc < 4; ++cc) {
+            float v[32];
+            const uint32_t ta = tmem + lane_off + TM_O + 128 * wg + cc * 32;
+            tmem_ld32(ta, v);
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] *= alpha;
-              tmem_st32(ta, v);
-            }
+            for (int j = 0; j < 32; ++j) v[j] *= alpha;
+            tmem_st32(ta, v);
           }
         }
         m2 = m_new;
       }
-      // P buffer n&1 is free once PV(n-2) completed
-      if (n >= 2)
-        t_ok = t_ok && __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE + (n & 1)),
-                                                         ((n - 2) >> 1) & 1, R.status));
-      uint8_t* prow = smem + OFF_P + (n & 1) * kPBytes + h * 128;
       const float mref = m2 == -INFINITY ? 0.f : m2;  // all scores -inf: p = 0
       float lsum = 0.f;
+      uint32_t pw[16];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t w4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2(s[8 * c + 2 * e] - mref);
-          const float p1 = ex2(s[8 * c + 2 * e + 1] - mref);
-          w4[e] = pack_bf16(p0, p1);  // bf16 only as the MMA operand
-          lsum += p0 + p1;            // the denominator keeps fp32 probabilities
-        }
-        const int cc = 4 * wg + c;
-        if (t_ok)
-          *reinterpret_cast<uint4*>(prow + ((cc ^ (h & 7)) * 16)) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      for (int j = 0; j < 16; ++j) {
+        const float p0 = ex2(s_cur[2 * j] - mref);
+        const float p1 = ex2(s_cur[2 * j + 1] - mref);
+        pw[j] = pack_bf16(p0, p1);  // bf16 only as the MMA operand
+        lsum += p0 + p1;            // the denominator keeps fp32 probabilities
       }
+      if (t_ok) tmem_st16(tmem + lane_off + TM_P + 16 * wg, pw);
       l += lsum;
       if (!t_ok) *abort_flag = 1;  // seen by everyone at the next barrier reduction
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P: generic -> async proxy
-      tc_fence_before();  // orders a rescale's tcgen05.st before the next MMA
-      mbar_arrive(bar(B_PFULL + (n & 1)));
+      tc_fence_before();           // orders the P store (and a rescale) before the PV MMA
+      mbar_arrive(bar(B_PFULL));
+#pragma unroll
+      for (int j = 0; j < 32; ++j) s_cur[j] = s_nxt[j];
     }
     if (!ok) *abort_flag = 1;
     // combine the two warpgroups' denominators (the first barrier retires the
@@ -474,10 +560,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     l += hmax[(wg ^ 1) * kH + h];
     // final output: warpgroup wg writes columns 128wg .. 128wg+127 of this CTA's half
     bool have_o = ok && ntiles > 0;
-    if (have_o) {
-      const int m = ntiles - 1;
-      have_o = mbar_wait(bar(B_PVDONE + (m & 1)), (m >> 1) & 1, R.status);
-    }
+    if (have_o) have_o = mbar_wait(bar(B_PVDONE), (ntiles - 1) & 1, R.status);
     have_o = __all_sync(0xffffffffu, have_o);
     tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -592,16 +675,12 @@ dsa_status_t launch_attn_tc(const Rows& R, int32_t row0, int32_t nrows, const ui
     part_o = reinterpret_cast<float*>(ws);
     part_lse = part_o + (size_t)nrows * sp.nsplit * kH * kDV;
   }
-  CUtensorMap qmap;
-  if (!make_tmap_2d(&qmap, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, (uint64_t)R.n_q * kH, 64,
-                    kH))
-    return DSA_ERR_CUDA;
   if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
   const dim3 grid(2 * nrows * sp.nsplit);
-  attn_tc_kernel<<<grid, kThreads, kSmem, st>>>(qmap, kv, R, row0, idx, k, sm_scale * kLog2e,
-                                                sp, out, lse, part_o, part_lse);
+  attn_tc_kernel<<<grid, kThreads, kSmem, st>>>(q, kv, R, row0, idx, k, sm_scale * kLog2e, sp,
+                                                out, lse, part_o, part_lse);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (sp.nsplit > 1) {
     attn_combine_kernel<<<dim3(nrows, kH), 128, 0, st>>>(row0, sp.nsplit, part_o, part_lse, out,

@@ -14,6 +14,7 @@ enum : unsigned {
   kErrTimeout = 1u,     // a bounded wait ran out
   kErrBadOffsets = 2u,  // kv_offsets not monotone / out of range
   kErrBadIndex = 4u,    // an index outside [0, L_b) (other than -1)
+  kErrLayout = 8u,      // shared memory not laid out as a kernel requires
 };
 
 // Description of the query rows, passed by value to every kernel.
