@@ -152,14 +152,15 @@ size_t dsa_sparse_mla_attn_workspace_size(const dsa_layout_t* layout, int32_t k,
  * capture mode, code inside a framework whose memory pool owns the whole
  * device, or plug-ins that are handed tensors but no allocator.  This call
  * takes the same arguments as dsa_sparse_mla_attn minus the workspace: the
- * decode split partials go to a fixed 64 MiB array that the library owns
+ * decode split partials go to a fixed 36 MiB array that the library owns
  * on every GPU where it is loaded, held until the process exits.
- *  - Capacity: a call whose split plan needs more than 64 MiB of partials
- *    (128 heads x 513 floats per (query row, split) pair, so at most 255
- *    pairs) returns DSA_ERR_WORKSPACE without launching anything.  With
- *    k <= 2048 that is every batch except 128..147 query rows; 148 rows or
- *    more need no partials at all.  Shapes that do not run on the tensor
- *    cores need no scratch and are never refused for size.
+ *  - Capacity: a call whose split plan needs more than 36 MiB of partials
+ *    (128 heads x 513 floats per (query row, split) pair, so at most 143
+ *    pairs) returns DSA_ERR_WORKSPACE without launching anything.  Batches
+ *    of 74 query rows or more are not split and need no partials; below
+ *    that, with k <= 2048, only 72 and 73 rows (144 and 146 pairs) exceed
+ *    the array.  Shapes that do not run on the tensor cores need no
+ *    scratch and are never refused for size.
  *  - Nothing needs zeroing: every call writes each partial it later reads.
  *  - The array is shared by all calls on a device and keeps the last call's
  *    contents: calls whose executions overlap on the GPU (different streams,

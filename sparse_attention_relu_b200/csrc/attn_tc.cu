@@ -9,44 +9,45 @@
 // selected positions are scattered, so the gather must be efficient.)
 //
 // TMEM holds 128 lanes x 512 fp32 columns, exactly the size of the 128 x 512
-// output accumulator, leaving no room for the score tile.  Each query row
-// therefore runs on a 2-CTA cluster that splits both contractions without
-// duplicating work:
-//   CTA c computes the partial scores over its half of the 576-d contraction
-//   (dims 288c .. 288c+287) and the output for its half of the 512 value
-//   columns (256c .. 256c+255).
-// The two partial score tiles are summed through distributed shared memory
-// (IEEE addition commutes, so both CTAs hold bit-identical scores and make
-// identical softmax decisions).
+// output accumulator.  Each query row therefore runs on two CTAs, one per
+// half of the 512 value columns.  Both compute the full 576-d scores of every
+// tile (the QK product is done twice) and make identical softmax decisions;
+// nothing is exchanged between them.  Measured on B200 with 2-CTA clusters on
+// two SMs, distributed shared memory moves only 3-10 bytes/cycle per SM
+// (remote loads, remote stores and bulk copies alike), so exchanging a 32 KB
+// partial-score tile per 64 selected rows would cost more than recomputing
+// the 9.4 MFLOP of QK on the tensor cores.
 //
-// Per CTA: the gathered tile holds the 5 swizzle atoms (64 columns each)
-// 4c .. 4c+4 of 64 selected rows, fetched with 16-byte cp.async by 64
-// producer threads, one row each, written straight into the 128-byte
-// swizzled layout the MMA reads (an empty slot is zero-filled); 4 such
-// stages are in flight.  Measured on B200: one thread issuing TMA
-// tile::gather4 (4 rows per instruction) needs about 9.3K cycles per such
-// tile, the spread cp.async gather a fraction of it.
+// Per CTA:
+//   TMEM columns   0..191  query dims 0..383 of every head (bf16 pairs, the
+//                          .ts MMA form reads A from TMEM)
+//                192..255  the 64-column score tile (fp32)
+//                256..511  this CTA's 256 output columns (fp32)
+//   shared memory: query dims 384..575 (three 128-byte-swizzled K-major
+//   atoms), two stages of 64 gathered cache rows (nine atoms of 64 dims,
+//   K-major for QK, MN-major for PV), and the tile's probabilities P (bf16,
+//   K-major) for PV.
+// The gather: 192 producer threads fetch the selected rows with 16-byte
+// cp.async, eight lanes per 128-byte segment, straight into the swizzled
+// layout the MMA reads (an empty slot -1 is zero-filled).  Measured on B200
+// (scattered rows, L2-resident source): cp.async sustains about 16 B/cycle
+// per SM from 2 producer warps, 30 from 4 and 40 from 16 -- a warp keeps a
+// bounded number of bytes in flight -- while one thread issuing TMA
+// tile::gather4 (4 rows per instruction) manages about 4.
 //
-// Both products take their A operand from TMEM (the .ts form), so shared
-// memory holds only gathered rows and the exchange buffers:
-//   columns   0..143  the CTA's 288 query dims of every head, bf16 pairs
-//   columns 160..223  the 64-column partial score tile (fp32)
-//   columns 224..255  P, the tile's probabilities as bf16 pairs
-//   columns 256..511  the 256-column output accumulator
-//
-// Warp roles (352 threads per CTA):
-//   warps 0-1  gather producer (indices -> shared memory, cp.async rows)
-//   warp 2     TMEM allocator and MMA issuer (one thread, issues whichever of
-//              QK(next tile) and PV(oldest tile with P ready) can go)
-//   warps 3-10 softmax, two warpgroups: a thread owns one head (its TMEM lane)
-//              and half of each tile's 64 rows.  Software-pipelined: tile
-//              n+1's partial scores leave for the peer before tile n's
-//              softmax runs (double-buffered exchange).  Online softmax in
-//              the log2 domain with a lazy rescale (the reference max moves
-//              only when a new score exceeds it by more than 2^8), P to TMEM
-//              as bf16, final normalisation and store.
-// Decode rows are split over several clusters; each writes a normalised
-// partial output and its log-sum-exp, merged by attn_combine_kernel.
+// Warp roles (480 threads per CTA):
+//   warps 0-5   gather producer (indices -> shared memory, cp.async rows)
+//   warp 6      TMEM allocator and MMA issuer (one thread, issues whichever of
+//               QK(next tile) and PV(oldest tile with P ready) can go)
+//   warps 7-14  softmax, two warpgroups: a thread owns one head (its TMEM
+//               lane) and half of each tile's 64 rows.  Online softmax in the
+//               log2 domain with a lazy rescale (the reference max moves only
+//               when a new score exceeds it by more than 2^8); P to shared
+//               memory as bf16; the denominator sums the fp32 probabilities;
+//               final normalisation and store of this CTA's output columns.
+// Decode rows are split over several CTA pairs; each split writes a
+// normalised partial output and its log-sum-exp, merged by
+// attn_combine_kernel.
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
@@ -59,31 +60,44 @@ using namespace sm100;
 namespace {
 
 constexpr int kH = 128, kDK = 576, kDV = 512;
-constexpr int kNT = 64;         // selected rows per tile
-constexpr int kProducers = 64;  // warps 0-1
-constexpr int kSoftmax0 = 96;   // first softmax thread (warps 3-10)
+constexpr int kNT = 64;                        // selected rows per tile
+constexpr int kAtoms = kDK / 64;               // 9 swizzle atoms per gathered row
+constexpr int kProducers = 192;                // warps 0-5
+constexpr int kMmaWarp = 6;
+constexpr int kSoftmax0 = 224;                 // first softmax thread (warps 7-14)
 constexpr int kSoftmaxThreads = 256;
-constexpr int kThreads = kSoftmax0 + kSoftmaxThreads;  // 352
-constexpr int kAtoms = 5;       // 64-column atoms held per CTA
-constexpr int kCBytes = kAtoms * kNT * 128;   // 40960 per stage
-constexpr int kStages = 4;
-constexpr int kXBytes = kH * kNT * 4;         // 32768 per exchange buffer
+constexpr int kThreads = kSoftmax0 + kSoftmaxThreads;  // 480
+constexpr int kAtomBytes = kNT * 128;          // 8192: one 64-dim atom of a tile
+constexpr int kCBytes = kAtoms * kAtomBytes;   // 73728 per stage
+constexpr int kStages = 2;
+// A stage is filled and released in two groups of atoms: the 5 atoms only QK
+// reads (group A, free once the QK steps over them retire) and the 4 atoms of
+// this CTA's value columns (group V, read by QK and PV, free once PV retires).
+constexpr int kAtomsA = 5, kAtomsV = 4;
+constexpr int kChunksA = kNT * kAtomsA * 8;    // 2560 16-byte chunks
+constexpr int kChunksV = kNT * kAtomsV * 8;    // 2048
+constexpr int kIdxRing = 4;                    // tiles whose indices are held
+constexpr int kQTmemDims = 384;                // query dims held in TMEM
+constexpr int kQSmemAtoms = (kDK - kQTmemDims) / 64;  // 3 atoms in shared memory
+constexpr int kQAtomBytes = kH * 128;          // 16384
+constexpr int kPBytes = kH * 128;              // P: 128 heads x 64 rows bf16
 constexpr int OFF_C = 0;
-constexpr int OFF_X = OFF_C + kStages * kCBytes;         // [2] exchange buffers
-constexpr int OFF_IDX = OFF_X + 2 * kXBytes;             // [stage][64] int32
-constexpr int OFF_MASK = OFF_IDX + kStages * kNT * 4;    // [stage][2] uint32 validity bits
-constexpr int OFF_HMAX = OFF_MASK + kStages * 2 * 4;     // [2 warpgroups][128] float
-constexpr int OFF_BAR = OFF_HMAX + 2 * kH * 4;
-constexpr int kNumBars = 20;
+constexpr int OFF_Q = OFF_C + kStages * kCBytes;
+constexpr int OFF_P = OFF_Q + kQSmemAtoms * kQAtomBytes;
+constexpr int OFF_IDX = OFF_P + kPBytes;                 // [ring][64] int32
+constexpr int OFF_MASK = OFF_IDX + kIdxRing * kNT * 4;   // [ring][2] uint32 validity bits
+constexpr int OFF_HMAX = OFF_MASK + kIdxRing * 2 * 4;    // [2 tiles][2 warpgroups][128] float
+constexpr int OFF_BAR = OFF_HMAX + 2 * 2 * kH * 4;
+constexpr int kNumBars = 16;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 // The dynamic window starts 1024-aligned (right after the driver's reserved
 // kilobyte, with no static shared memory); the kernel checks it.
 constexpr int kSmem = OFF_MISC + 16;
 static_assert(kSmem <= 232448, "shared memory");
+static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0 && OFF_BAR % 8 == 0, "alignment");
 // TMEM columns
-constexpr uint32_t TM_Q = 0;     // the CTA's 288 query dims of all heads, bf16 pairs (144 cols)
-constexpr uint32_t TM_S = 160;   // 64-column score tile
-constexpr uint32_t TM_P = 224;   // 32-column bf16 P tile (the PV A operand)
+constexpr uint32_t TM_Q = 0;     // query dims 0..383 of all heads, bf16 pairs (192 cols)
+constexpr uint32_t TM_S = 192;   // 64-column score tile
 constexpr uint32_t TM_O = 256;   // 256-column output accumulator
 constexpr uint32_t IDESC_QK = idesc(1, 128, kNT);
 constexpr uint32_t IDESC_PV = idesc(1, 128, 256, false, true);
@@ -92,64 +106,19 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;  // log2 headroom before the reference max moves
 
 enum {
-  B_QREADY = 0,  // the query is in TMEM (every softmax thread)
-  B_CFULL = 1,   // [4] stage rows landed (producers)
-  B_CEMPTY = 5,  // [4] PV of the stage retired
-  B_SFULL = 9,   // QK retired
-  B_SEMPTY = 10, // scores read (every softmax thread)
-  B_PFULL = 11,  // P stored in TMEM (every softmax thread)
-  B_PVDONE = 12, // PV retired
-  B_XFULL = 13,  // [2] the peer's partial scores arrived
-  B_XEMPTY = 15, // [2] the peer read our partial scores
-  B_DRAIN = 17
+  B_QREADY = 0,   // the query is in TMEM and shared memory (every softmax thread)
+  B_AFULL = 1,    // [2] group-A rows landed, indices published (producers)
+  B_VFULL = 3,    // [2] group-V rows landed (producers)
+  B_AEMPTY = 5,   // [2] QK steps over group A retired
+  B_VEMPTY = 7,   // [2] PV of the stage retired
+  B_SFULL = 9,    // QK retired
+  B_SEMPTY = 10,  // scores read (every softmax thread)
+  B_PFULL = 11,   // P stored (every softmax thread)
+  B_PVDONE = 12,  // PV retired
+  B_DRAIN = 13
 };
+static_assert(B_DRAIN < kNumBars, "barrier count");
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
-               ::: "memory");
-}
-__device__ __forceinline__ uint32_t map_peer(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-__device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-__device__ __forceinline__ bool try_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.b32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait with cluster-scope acquire (data written by the peer CTA).
-__device__ __forceinline__ bool wait_cluster(uint32_t bar, uint32_t parity, unsigned* status) {
-  if (try_cluster(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!try_cluster(bar, parity)) {
-    if (clock64() - t0 > kSpinLimit) {
-      atomicOr(status, kErrTimeout);
-      return false;
-    }
-  }
-  return true;
-}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -178,16 +147,6 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8])
       "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n\t"
       "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-      "r"(v[15])
       : "memory");
 }
 
@@ -219,13 +178,21 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&p);
 }
 
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads (the MMA reading the query and P operands).
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 struct Split {
   int nsplit, tiles_per_split;
 };
 
+// Decode rows are few: split each row's tiles so that the CTA pairs cover
+// the 148 SMs (two CTAs per pair, one CTA per SM).
 __host__ __device__ inline Split plan_split(int32_t nrows, int k) {
   const int tiles = (k + kNT - 1) / kNT;
-  int want = nrows >= 148 ? 1 : (148 + nrows - 1) / nrows;
+  int want = nrows >= 74 ? 1 : (74 + nrows - 1) / nrows;
   if (want > tiles) want = tiles;
   if (want < 1) want = 1;
   Split s;
@@ -234,7 +201,7 @@ __host__ __device__ inline Split plan_split(int32_t nrows, int k) {
   return s;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kv, Rows R,
                    int32_t row0, const int32_t* __restrict__ idx, int k, float scale2, Split sp,
                    uint16_t* __restrict__ out, float* __restrict__ lse,
@@ -244,7 +211,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   if (sb & 1023u) {  // the swizzled operand layouts need 1024-byte alignment
     if (threadIdx.x == 0) raise_status(R, kErrLayout);
-    return;  // uniform across the cluster: both CTAs share the layout
+    return;
   }
   int32_t* sidx = reinterpret_cast<int32_t*>(smem + OFF_IDX);
   uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + OFF_MASK);
@@ -254,7 +221,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t crank = cluster_rank(), peer = crank ^ 1u;
+  const int half = blockIdx.x & 1;  // this CTA's output columns 256*half ..
   const int item = blockIdx.x >> 1;
   const int32_t rloc = item / sp.nsplit, split = item % sp.nsplit;
   const int32_t r = row0 + rloc;
@@ -266,34 +233,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(bar(B_QREADY), kSoftmaxThreads);
     for (int i = 0; i < kStages; ++i) {
-      // per producer: a release-arrive after its index store and a cp.async arrive
-      mbar_init(bar(B_CFULL + i), 2 * kProducers);
-      mbar_init(bar(B_CEMPTY + i), 1);
+      // per producer: an arrive after the index store and a cp.async arrive
+      mbar_init(bar(B_AFULL + i), 2 * kProducers);
+      mbar_init(bar(B_VFULL + i), kProducers);  // a cp.async arrive per producer
+      mbar_init(bar(B_AEMPTY + i), 1);
+      mbar_init(bar(B_VEMPTY + i), 1);
     }
     mbar_init(bar(B_SFULL), 1);
     mbar_init(bar(B_SEMPTY), kSoftmaxThreads);
     mbar_init(bar(B_PFULL), kSoftmaxThreads);
     mbar_init(bar(B_PVDONE), 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(B_XFULL + i), 1);  // one release-arrive from the peer per tile
-      mbar_init(bar(B_XEMPTY + i), 1);
-    }
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 2) {
+  if (warp == kMmaWarp) {
     tmem_alloc(sb + OFF_MISC, 512);
     tmem_relinquish();
   }
   tc_fence_before();
-  cluster_sync();  // barriers of both CTAs initialised before any remote arrive
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 2) {
+  if (warp < kMmaWarp) {
     // ------------------------------------------------------------ gather producer
-    const uint16_t* kvb = kv + ri.kbase * kDK + 256 * crank;  // atoms 4c .. 4c+4
+    const char* kvb = reinterpret_cast<const char*>(kv + ri.kbase * kDK);
     auto load_idx = [&](int n) -> int32_t {
       const int slot = slot_lo + n * kNT + tid;
       int32_t s = slot < slot_hi ? __ldg(idx + (int64_t)rloc * k + slot) : -1;
@@ -303,51 +268,98 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       return s;
     };
-    // A warp instruction copies 4 rows x 128 contiguous bytes: lanes 8g..8g+7
-    // take the 16-byte chunks of row 4j+g of this warp's 32 rows.
-    const int sub = lane >> 3, ch = lane & 7;
-    int32_t pre = ntiles > 0 ? load_idx(0) : -1;
+    // Threads 0..63 own the index of tile row tid.
+    int32_t pre = (tid < kNT && ntiles > 0) ? load_idx(0) : -1;
+    // Issues 16-byte chunk i of group G (eight lanes per 128-byte segment of
+    // a row, a warp four consecutive segments) of tile n into stage st.
+    auto issue = [&](int st, int ring, int i, bool group_a) {
+      const int ch = i & 7, seg = i >> 3;
+      int row, atom;
+      if (group_a) {  // the five atoms only QK reads
+        row = seg / kAtomsA;
+        const int ai = seg - row * kAtomsA;
+        atom = ai < 4 ? 4 * (half ^ 1) + ai : 8;
+      } else {  // this CTA's value columns
+        row = seg >> 2;
+        atom = 4 * half + (seg & 3);
+      }
+      const int32_t s = sidx[ring * kNT + row];
+      const char* src = s >= 0 ? kvb + (int64_t)s * (kDK * 2) + atom * 128 + ch * 16
+                               : reinterpret_cast<const char*>(kv);
+      const uint32_t nbytes = s >= 0 ? 16u : 0u;  // 0: zero-fill
+      const uint32_t dst = sb + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128 +
+                           ((uint32_t)(ch ^ (row & 7)) << 4);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                   "r"(nbytes)
+                   : "memory");
+    };
     for (int n = 0; n < ntiles; ++n) {
-      const int st = n % kStages;
-      const bool ok = mbar_wait(bar(B_CEMPTY + st), ((n / kStages) & 1) ^ 1, R.status) &&
-                      !*abort_flag;
+      const int st = n % kStages, ring = n % kIdxRing;
+      const uint32_t par = ((n / kStages) & 1) ^ 1;
+      // group A of the stage is free once QK(n-2) read it
+      bool ok = mbar_wait(bar(B_AEMPTY + st), par, R.status) && !*abort_flag;
       if (!bar_and<2, kProducers>(ok)) {
         *abort_flag = 1;
         break;
       }
-      sidx[st * kNT + tid] = pre;
-      const uint32_t bits = __ballot_sync(0xffffffffu, pre >= 0);
-      if (lane == 0) vmask[st * 2 + warp] = bits;
-      mbar_arrive(bar(B_CFULL + st));  // publishes indices and mask to the softmax threads
-      asm volatile("bar.sync 2, 64;" ::: "memory");  // every producer sees the tile's indices
-      pre = n + 1 < ntiles ? load_idx(n + 1) : -1;    // overlaps the copies below
-      const uint32_t cb = sb + OFF_C + st * kCBytes;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int row = warp * 32 + 4 * j + sub;
-        const int32_t s = sidx[st * kNT + row];
-        const char* src = reinterpret_cast<const char*>(s >= 0 ? kvb + (int64_t)s * kDK : kv);
-        const uint32_t nbytes = s >= 0 ? 16u : 0u;  // 0: zero-fill
-        const uint32_t dst = cb + row * 128 + ((uint32_t)(ch ^ (row & 7)) << 4);
-#pragma unroll
-        for (int la = 0; la < kAtoms; ++la)
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst + la * kNT * 128),
-                       "l"(src + (la * 64 + ch * 8) * 2), "r"(nbytes)
-                       : "memory");
+      if (tid < kNT) {
+        sidx[ring * kNT + tid] = pre;
+        const uint32_t bits = __ballot_sync(0xffffffffu, pre >= 0);
+        if (lane == 0) vmask[ring * 2 + warp] = bits;
       }
-      // arrives on the stage barrier once this thread's copies have landed
-      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_CFULL + st))
+      mbar_arrive(bar(B_AFULL + st));  // publishes indices and mask to the softmax threads
+      asm volatile("bar.sync 2, %0;" ::"n"(kProducers) : "memory");  // producers see the indices
+      if (tid < kNT) pre = n + 1 < ntiles ? load_idx(n + 1) : -1;  // overlaps the copies below
+#pragma unroll
+      for (int j = 0; j < (kChunksA + kProducers - 1) / kProducers; ++j)
+        if (tid + kProducers * j < kChunksA) issue(st, ring, tid + kProducers * j, true);
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_AFULL + st))
+                   : "memory");
+      // group V of the stage is free once PV(n-2) retired
+      ok = mbar_wait(bar(B_VEMPTY + st), par, R.status) && !*abort_flag;
+      if (!bar_and<2, kProducers>(ok)) {
+        *abort_flag = 1;
+        break;
+      }
+#pragma unroll
+      for (int j = 0; j < (kChunksV + kProducers - 1) / kProducers; ++j)
+        if (tid + kProducers * j < kChunksV) issue(st, ring, tid + kProducers * j, false);
+      // arrives on the barrier once this thread's copies (groups A and V) have landed
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_VFULL + st))
                    : "memory");
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == 2) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(bar(B_QREADY), 0, R.status);
-      // Issue whichever is ready: QK of the next tile (rows landed, score
-      // tile free) or PV of the oldest tile whose P is in TMEM.  PV never
-      // waits for a later tile's rows.
-      int nq = 0, np = 0;
+      // Three kinds of work, issued as soon as they can go (PV first):
+      //   QK-A(n): the 20 K steps over group A (rows landed, score tile free)
+      //   QK-B(n): the 16 K steps over group V, then S(n) is complete
+      //   PV(n):   P(n) stored
+      // Splitting QK lets PV(n-1) slip in between QK-A(n) and QK-B(n), and
+      // group A of a stage is released as soon as its QK steps retire.
+      // Polling uses the non-blocking test: try_wait may suspend the thread
+      // while another of the three could already go.
+      int na = 0, nb = 0, np = 0;
+      // Descriptors advance by adding byte offsets / 16 to the start address
+      // field (no carry: shared addresses stay below 256 KB).
+      const uint64_t dq0 = desc_sw128(sb + OFF_Q, 1024);
+      const uint64_t dp0 = desc_sw128(sb + OFF_P, 1024);
+      const uint32_t ts = tmem + TM_S;
+      // One QK K step over dims 64*atom + 16*sub of the stage whose
+      // descriptor is db: A from TMEM for dims < 384, else from the query
+      // atoms in shared memory.  `atom` and `sub` are compile-time after
+      // unrolling, so a step is a handful of instructions.
+      auto qk_step = [&](uint64_t db, int atom, int sub, uint32_t acc) {
+        const uint64_t bdesc = db + (uint64_t)((atom * kAtomBytes + sub * 32) >> 4);
+        if (atom < kQTmemDims / 64)
+          mma_bf16_ts(ts, tmem + TM_Q + 32 * atom + 8 * sub, bdesc, IDESC_QK, acc);
+        else
+          mma_bf16(ts,
+                   dq0 + (uint64_t)(((atom - kQTmemDims / 64) * kQAtomBytes + sub * 32) >> 4),
+                   bdesc, IDESC_QK, acc);
+      };
       long long t0 = clock64();
       while (ok && np < ntiles) {
         if (*abort_flag) {
@@ -355,39 +367,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           break;
         }
         bool progressed = false;
-        if (nq < ntiles) {
-          const int st = nq % kStages;
-          if (mbar_try(bar(B_CFULL + st), (nq / kStages) & 1) &&
-              mbar_try(bar(B_SEMPTY), (nq & 1) ^ 1)) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // cp.async rows
-            tc_fence_after();
-            const uint32_t cb = sb + OFF_C + st * kCBytes;
+        if (np < nb && mbar_test(bar(B_PFULL), np & 1)) {
+          tc_fence_after();
+          // this CTA's value columns: atoms 4*half .. 4*half+3 of the stage
+          const uint64_t dv = desc_sw128_mn(
+              sb + OFF_C + (np % kStages) * kCBytes + 4 * half * kAtomBytes, kAtomBytes, 1024);
 #pragma unroll
-            for (int kk = 0; kk < 18; ++kk) {
-              const int e = 288 * (int)crank + 16 * kk;  // global contraction index
-              const int la = e / 64 - 4 * (int)crank, off = (e % 64) * 2;
-              mma_bf16_ts(tmem + TM_S, tmem + TM_Q + 8 * kk,
-                          desc_sw128(cb + la * kNT * 128 + off, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(bar(B_SFULL));
-            ++nq;
-            progressed = true;
-          }
-        }
-        if (np < nq) {
-          if (mbar_try(bar(B_PFULL), np & 1)) {
-            tc_fence_after();
-            const uint32_t cb = sb + OFF_C + (np % kStages) * kCBytes;  // stage of tile np
+          for (int kk = 0; kk < kNT / 16; ++kk)
+            mma_bf16(tmem + TM_O, dp0 + (uint64_t)(kk * 2), dv + (uint64_t)(kk * 128), IDESC_PV,
+                     (np > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(B_PVDONE));
+          mma_commit(bar(B_VEMPTY + np % kStages));
+          ++np;
+          progressed = true;
+        } else if (nb < na && mbar_test(bar(B_VFULL + nb % kStages), (nb / kStages) & 1)) {
+          fence_async_smem();  // rows written by cp.async (generic proxy)
+          tc_fence_after();
+          const uint64_t db = desc_sw128(sb + OFF_C + (nb % kStages) * kCBytes, 1024);
+          if (half) {
 #pragma unroll
-            for (int kk = 0; kk < kNT / 16; ++kk)
-              mma_bf16_ts(tmem + TM_O, tmem + TM_P + kk * 8,
-                          desc_sw128_mn(cb + kk * 2048, kNT * 128, 1024), IDESC_PV,
-                          (np > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(bar(B_PVDONE));
-            mma_commit(bar(B_CEMPTY + np % kStages));
-            ++np;
-            progressed = true;
+            for (int a = 0; a < kAtomsV; ++a)
+#pragma unroll
+              for (int sub = 0; sub < 4; ++sub) qk_step(db, 4 + a, sub, 1u);
+          } else {
+#pragma unroll
+            for (int a = 0; a < kAtomsV; ++a)
+#pragma unroll
+              for (int sub = 0; sub < 4; ++sub) qk_step(db, a, sub, 1u);
           }
+          mma_commit(bar(B_SFULL));
+          ++nb;
+          progressed = true;
+        } else if (na == nb && na < ntiles &&
+                   mbar_test(bar(B_AFULL + na % kStages), (na / kStages) & 1) &&
+                   mbar_test(bar(B_SEMPTY), (na & 1) ^ 1)) {
+          fence_async_smem();  // rows written by cp.async (generic proxy)
+          tc_fence_after();
+          const uint64_t db = desc_sw128(sb + OFF_C + (na % kStages) * kCBytes, 1024);
+          // group A atoms: the other latent half (4*(half^1) .. +3), then rotary (8)
+          if (half) {
+#pragma unroll
+            for (int a = 0; a < kAtomsA; ++a)
+#pragma unroll
+              for (int sub = 0; sub < 4; ++sub)
+                qk_step(db, a < 4 ? a : 8, sub, (a > 0 || sub > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int a = 0; a < kAtomsA; ++a)
+#pragma unroll
+              for (int sub = 0; sub < 4; ++sub)
+                qk_step(db, a < 4 ? 4 + a : 8, sub, (a > 0 || sub > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(B_AEMPTY + na % kStages));
+          ++na;
+          progressed = true;
         }
         if (progressed) {
           t0 = clock64();
@@ -405,30 +438,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax
     // Two warpgroups; warpgroup wg handles rows 32wg .. 32wg+31 of every
-    // tile for the head of its TMEM lane.  Software-pipelined: the partial
-    // scores of tile n+1 go to the peer before tile n's softmax runs, so the
-    // exchange overlaps the arithmetic (double-buffered exchange buffers).
-    const int wg = (warp - 3) >> 2;
+    // tile for the head of its TMEM lane.
+    const int wg = (warp - kSoftmax0 / 32) >> 2;
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    // The query: this CTA's 288 contraction dims of head h, as bf16 pairs in
-    // TMEM columns TM_Q .. TM_Q+143 (warpgroup wg stores 72 of them).
+    const uint16_t* qrow = q + ((int64_t)r * kH + h) * kDK;
     {
-      const uint4* qsrc = reinterpret_cast<const uint4*>(
-          q + ((int64_t)r * kH + h) * kDK + 288 * crank + 144 * wg);
+      // query dims 0..383 -> TMEM columns 0..191 (warpgroup wg: 192 dims)
 #pragma unroll
-      for (int part = 0; part < 3; ++part) {  // 3 x 48 dims = 3 x 24 columns
+      for (int part = 0; part < 4; ++part) {  // 4 x 48 dims = 4 x 24 columns
+        const uint4* qs = reinterpret_cast<const uint4*>(qrow + 192 * wg + 48 * part);
         uint32_t w24[24];
 #pragma unroll
         for (int v = 0; v < 6; ++v) {
-          const uint4 x = __ldg(qsrc + part * 6 + v);
+          const uint4 x = __ldg(qs + v);
           w24[4 * v] = x.x;
           w24[4 * v + 1] = x.y;
           w24[4 * v + 2] = x.z;
           w24[4 * v + 3] = x.w;
         }
-        const uint32_t ta = tmem + lane_off + TM_Q + 72 * wg + 24 * part;
+        const uint32_t ta = tmem + lane_off + TM_Q + 96 * wg + 24 * part;
         uint32_t a8[8], b8[8], c8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -440,82 +470,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_st8(ta + 8, b8);
         tmem_st8(ta + 16, c8);
       }
+      // query dims 384..575 -> three K-major atoms in shared memory (row h;
+      // warpgroup wg stores 16-byte chunks 12wg .. 12wg+11 of the 24)
+#pragma unroll
+      for (int c = 0; c < 12; ++c) {
+        const int chunk = 12 * wg + c, a = chunk >> 3, ch = chunk & 7;
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(qrow + kQTmemDims + 8 * chunk));
+        *reinterpret_cast<uint4*>(smem + OFF_Q + a * kQAtomBytes + h * 128 +
+                                  ((ch ^ (h & 7)) << 4)) = x;
+      }
+      fence_async_smem();
       tc_fence_before();
       mbar_arrive(bar(B_QREADY));
     }
-    const uint32_t xrow_peer0 = map_peer(sb + OFF_X + h * (kNT * 4), peer);
-    const uint32_t xfull_peer0 = map_peer(bar(B_XFULL), peer);
-    const uint32_t xempty_peer0 = map_peer(bar(B_XEMPTY), peer);
+    // row h of P: this warpgroup's 32 rows are 16-byte chunks 4wg .. 4wg+3
+    uint8_t* const prow = smem + OFF_P + h * 128;
     float m2 = -INFINITY, l = 0.f;
     bool ok = true;
-    float s_cur[32], s_nxt[32];
-    // Loads tile m's partial scores into d and ships them to the peer.
-    auto send = [&](int m, float (&d)[32]) -> bool {
-      const int st = m % kStages, xb = m & 1;
+    for (int n = 0; ok && n < ntiles; ++n) {
+      const int st = n % kStages;
+      float s[32];
+      // the tile's validity bits were published with its group A
       bool w_ok = __all_sync(0xffffffffu,
-                             mbar_wait(bar(B_CFULL + st), (m / kStages) & 1, R.status) &&
-                                 mbar_wait(bar(B_SFULL), m & 1, R.status) && !*abort_flag);
+                             mbar_wait(bar(B_AFULL + st), (n / kStages) & 1, R.status) &&
+                                 mbar_wait(bar(B_SFULL), n & 1, R.status) && !*abort_flag);
       if (w_ok) {
         tc_fence_after();
-        tmem_ld32(tmem + lane_off + TM_S + 32 * wg, d);
+        tmem_ld32(tmem + lane_off + TM_S + 32 * wg, s);
         tc_fence_before();
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) d[j] = 0.f;
+        for (int j = 0; j < 32; ++j) s[j] = 0.f;
       }
-      mbar_arrive(bar(B_SEMPTY));
-      w_ok = w_ok && __all_sync(0xffffffffu, mbar_wait(bar(B_XEMPTY + xb), ((m >> 1) & 1) ^ 1,
-                                                       R.status));
-      if (w_ok) {
-        const uint32_t xr = xrow_peer0 + xb * kXBytes;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int cc = 8 * wg + c;
-          st_cluster_v4(xr + ((cc ^ (h & 7)) * 16), d[4 * c], d[4 * c + 1], d[4 * c + 2],
-                        d[4 * c + 3]);
-        }
-      }
-      if (!bar_and<1, kSoftmaxThreads>(w_ok)) return false;  // all stores issued
-      if (tid == kSoftmax0) arrive_remote(xfull_peer0 + 8u * xb);  // one cumulative release
-      return true;
-    };
-    if (ntiles > 0) ok = send(0, s_cur);
-    for (int n = 0; ok && n < ntiles; ++n) {
-      const int st = n % kStages, xb = n & 1;
-      if (n + 1 < ntiles && !send(n + 1, s_nxt)) {
-        ok = false;
-        break;
-      }
-      // the peer's half of tile n
-      bool w_ok = __all_sync(0xffffffffu, wait_cluster(bar(B_XFULL + xb), (n >> 1) & 1, R.status));
-      const uint32_t bits = vmask[st * 2 + wg];
+      const uint32_t bits = vmask[(n % kIdxRing) * 2 + wg];
+      mbar_arrive(bar(B_SEMPTY));  // the MMA may overwrite the score tile
       float hm = -INFINITY;
-      {
-        const float4* xr = reinterpret_cast<const float4*>(smem + OFF_X + xb * kXBytes +
-                                                            h * (kNT * 4));
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int cc = 8 * wg + c;
-          const float4 v = w_ok ? xr[cc ^ (h & 7)] : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 4 * c + e;
-            s_cur[j] = ((bits >> j) & 1u) ? (s_cur[j] + vv[e]) * scale2 : -INFINITY;
-            hm = fmaxf(hm, s_cur[j]);
-          }
-        }
+      for (int j = 0; j < 32; ++j) {
+        s[j] = ((bits >> j) & 1u) ? s[j] * scale2 : -INFINITY;
+        hm = fmaxf(hm, s[j]);
       }
-      hmax[wg * kH + h] = hm;
-      if (!bar_and<1, kSoftmaxThreads>(w_ok)) {  // exchange buffer read, half maxima visible
+      float* const hm_buf = hmax + (n & 1) * (2 * kH);  // two tiles in flight
+      hm_buf[wg * kH + h] = hm;
+      if (!bar_and<1, kSoftmaxThreads>(w_ok)) {  // half maxima visible
         ok = false;
         break;
       }
-      if (tid == kSoftmax0) arrive_remote(xempty_peer0 + 8u * xb);
-      const float mt = fmaxf(hm, hmax[(wg ^ 1) * kH + h]);  // same value in both warpgroups
+      const float mt = fmaxf(hm, hm_buf[(wg ^ 1) * kH + h]);  // same value in both warpgroups
       // P of tile n-1 is consumed and O is final up to tile n-1 once PV(n-1) retired
-      bool t_ok = n == 0 || __all_sync(0xffffffffu,
-                                       mbar_wait(bar(B_PVDONE), (n - 1) & 1, R.status));
+      const bool t_ok = n == 0 || __all_sync(0xffffffffu,
+                                             mbar_wait(bar(B_PVDONE), (n - 1) & 1, R.status));
       if (mt > m2 + kRescale || (m2 == -INFINITY && mt != -INFINITY)) {
         const float m_new = fmaxf(mt, m2);
         const float alpha = ex2(m2 - m_new);  // 0 when m2 = -inf
@@ -538,18 +542,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t pw[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const float p0 = ex2(s_cur[2 * j] - mref);
-        const float p1 = ex2(s_cur[2 * j + 1] - mref);
+        const float p0 = ex2(s[2 * j] - mref);
+        const float p1 = ex2(s[2 * j + 1] - mref);
         pw[j] = pack_bf16(p0, p1);  // bf16 only as the MMA operand
         lsum += p0 + p1;            // the denominator keeps fp32 probabilities
       }
-      if (t_ok) tmem_st16(tmem + lane_off + TM_P + 16 * wg, pw);
+      if (t_ok) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(prow + (((4 * wg + c) ^ (h & 7)) << 4)) =
+              make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+      }
       l += lsum;
       if (!t_ok) *abort_flag = 1;  // seen by everyone at the next barrier reduction
-      tc_fence_before();           // orders the P store (and a rescale) before the PV MMA
+      fence_async_smem();          // P stores before the PV MMA reads them
+      tc_fence_before();           // a rescale's TMEM stores before the PV MMA
       mbar_arrive(bar(B_PFULL));
-#pragma unroll
-      for (int j = 0; j < 32; ++j) s_cur[j] = s_nxt[j];
     }
     if (!ok) *abort_flag = 1;
     // combine the two warpgroups' denominators (the first barrier retires the
@@ -575,7 +583,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = 0.f;
       }
-      const int col = (int)crank * 256 + c32 * 32;
+      const int col = half * 256 + c32 * 32;
       if (final_out) {
         uint16_t* o = out + ((int64_t)r * kH + h) * kDV + col;
 #pragma unroll
@@ -593,7 +601,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                          v[4 * q4 + 2] * inv, v[4 * q4 + 3] * inv);
       }
     }
-    if (crank == 0 && wg == 0) {
+    if (half == 0 && wg == 0) {
       if (final_out) {
         if (lse) lse[(int64_t)r * kH + h] = lse_v;
       } else {
@@ -604,11 +612,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  cluster_sync();  // the peer may still write into our shared memory until here
 }
 
 // Merges split partials: out = sum_i exp(lse_i - lse) o_i, lse = log sum_i exp(lse_i).
@@ -648,8 +655,9 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(int32_t row0, int nsp
 }
 
 // Fixed scratch for callers that cannot allocate device memory (see
-// launch_attn_tc_static): the split partials of one call, 64 MiB.
-constexpr size_t kStaticScratchBytes = size_t(64) << 20;
+// launch_attn_tc_static): the split partials of one call, 36 MiB (143
+// (query row, split) blocks of 128 x 513 floats).
+constexpr size_t kStaticScratchBytes = size_t(36) << 20;
 static __device__ __align__(256) float g_attn_scratch[kStaticScratchBytes / sizeof(float)];
 
 }  // namespace

@@ -48,6 +48,21 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of the phase with the given parity (mbarrier.try_wait
+// may suspend the thread for a while when the phase is incomplete; a thread
+// that polls several barriers in turn must not be held up by one of them).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // kSpinLimit cycles, raising kErrTimeout in the status word; returns false.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status) {
@@ -113,7 +128,20 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t sbo) {
   return d;
 }
 
-// Same layout, MN-major (the contiguous 128-byte rows run along M/N):
+// K-major operand in the 64-byte-swizzled layout: rows of 64 bytes, 8-row
+// groups of 512 bytes, groups `sbo` bytes apart along M/N.  The tile base
+// must be 512-aligned; advancing K inside a row adds the byte offset.
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;                   // 64-byte swizzle
+  return d;
+}
+
+// Same layout as desc_sw128, MN-major (the contiguous 128-byte rows run along M/N):
 // `lbo` = bytes between 64-element (128 B) column blocks along M/N,
 // `sbo` = bytes between 8-row groups along K.
 __device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t saddr, uint32_t lbo, uint32_t sbo) {

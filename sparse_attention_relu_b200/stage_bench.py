@@ -5,7 +5,7 @@
 
 Small, fixed cases meant for profiler captures of a single kernel:
   attn/prefill   one sequence of T tokens (cache L2-resident); row t selects
-                 min(t+1, k) distinct positions spread over 0..t
+                 min(t+1, k) distinct random positions in 0..t
   attn/decode    64 sequences x 16384 tokens (cache from HBM), k scattered positions
   indexer|topk   e4m3 prefill of T tokens (the unit calls write full score rows)
 Prints one line with the last repetition's time and throughput.
@@ -41,10 +41,16 @@ def attn(case: str, reps: int, T: int, k: int = 2048):
         offs = torch.tensor([0, T], dtype=torch.int32, device=dev)
         lay = dsa.Layout(offs, dsa.DSA_PREFILL, T, T, T)
         n_q, n_k = T, T
-        t = torch.arange(T, device=dev)[:, None]
-        j = torch.arange(k, device=dev)[None, :]
-        stride = torch.clamp((t + 1) // k, min=1)
-        idx = torch.where(t + 1 <= k, torch.where(j <= t, j, -1), t - j * stride)
+        # the k best of random causal scores: scattered positions, as the
+        # indexer selects them
+        idx = torch.empty(T, k, dtype=torch.int64, device=dev)
+        pos = torch.arange(T, device=dev)
+        for r0 in range(0, T, 1024):
+            r1 = min(T, r0 + 1024)
+            sc = torch.rand(r1 - r0, T, device=dev)
+            sc.masked_fill_(pos[None, :] > pos[r0:r1, None], -1.0)
+            v, i = torch.topk(sc, k, dim=1)
+            idx[r0:r1] = torch.where(v >= 0, i, -1)
     else:
         B, L = 64, 16384
         offs = torch.arange(0, (B + 1) * L, L, dtype=torch.int32, device=dev)

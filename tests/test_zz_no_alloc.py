@@ -48,12 +48,12 @@ def test_noalloc_matches_workspace_call_twice(lens, k):
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch():
-    """128 decode rows at k = 2048 split in two: 256 partial blocks, one more
-    than the fixed scratch holds -> DSA_ERR_WORKSPACE, nothing launched."""
-    cfg = workloads.custom("decode", [64] * 128, idx_dtype="bf16", k=2048, seed=3)
+    """73 decode rows at k = 2048 split in two: 146 partial blocks, more than
+    the 143 the fixed scratch holds -> DSA_ERR_WORKSPACE, nothing launched."""
+    cfg = workloads.custom("decode", [64] * 73, idx_dtype="bf16", k=2048, seed=3)
     dev = Dev(workloads.generate(cfg))
-    idx = torch.full((128, 2048), -1, dtype=torch.int32, device="cuda")
-    out = torch.zeros(128, 128, 512, dtype=torch.bfloat16, device="cuda")
+    idx = torch.full((73, 2048), -1, dtype=torch.int32, device="cuda")
+    out = torch.zeros(73, 128, 512, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(dsa.DSAError) as e:
         dsa.dsa_sparse_mla_attn_noalloc(dev.layout, dev.d.q, dev.d.kv, idx, 2048, 512,
                                         cfg.sm_scale, out)
