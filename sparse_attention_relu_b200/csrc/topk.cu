@@ -5,14 +5,27 @@
 // figure): the cut-off is the k-th best score.  Ties go to the lower
 // position; -0 == +0; NaN ranks as -inf.
 //
-// One CTA owns a row.  Scores become 32-bit keys whose unsigned order is
-// the float order.  Three histogram passes (11 + 11 + 10 bits) pin down the
-// exact key tau of the k-th best element and the number c_gt of elements
-// strictly above it; a final pass writes every element above tau (any
-// order) and the first k - c_gt elements equal to tau in position order,
-// the latter through a block-wide ordered compaction (ballot + warp prefix
-// + a scan of warp totals).  When the row fits, the first pass parks the
-// keys in shared memory and the later passes never touch global memory.
+// One CTA of 512 threads owns a row, and several CTAs share an SM (about
+// 25 KB of shared memory each) so that one row's reads overlap another's
+// arithmetic.  Scores become 32-bit keys whose unsigned order is the float
+// order, and the row is read twice (the second time from L2):
+//   pass 1  a 2048-bin histogram fixes the bin b1 that holds the k-th best
+//           score.  A bin is the sign and 32 steps per binade of the
+//           magnitude over 2^-16 .. 2^16 (saturating outside): monotone, so a
+//           higher bin means a strictly larger score, and indexer scores,
+//           which crowd a few binades, spread over hundreds of bins instead
+//           of the few dozen that the top bits of the fp32 key would give
+//           (the histogram atomics would serialise on them);
+//   pass 2  b1 is an interval [lo, hi] of floats: every score above hi is
+//           written out at once (in any order), the members of b1 --
+//           typically a hundred or so -- go to a candidate buffer in shared
+//           memory with their fp32 keys.
+// The candidates are then ranked directly (key, then position: ties go to
+// the lower position) and the best k - |above b1| of them written out.  A
+// bin b1 with more members than the buffer holds is resolved by radix
+// passes over the row instead (11 + 11 + 10 bits of the fp32 key), with
+// ties at the cut filled from the lowest positions by an ordered pass over
+// the row (ballot + warp prefix + a scan of warp totals).
 #include "kernels.cuh"
 
 namespace dsa {
@@ -22,8 +35,7 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
-// Largest row cached in shared memory (keys): 48K entries = 192 KB.
-constexpr int kCacheCap = 48 * 1024;
+constexpr int kCand = 2048;  // candidate buffer (keys + positions)
 
 __device__ __forceinline__ uint32_t rank_key(float x) {
   uint32_t u = __float_as_uint(x);
@@ -32,12 +44,39 @@ __device__ __forceinline__ uint32_t rank_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Bin of a score, 0 .. 2047, non-decreasing in the score: the magnitude
+// bits >> 18 are (exponent, top 5 mantissa bits), clamped to the 1024 steps
+// of 2^-16 .. 2^16; negative scores mirror below 1024.  -0 counts as +0 and
+// NaN as -inf (bin 0).
+constexpr int kMagBase = (111 << 5);  // exponent 111 = 2^-16, mantissa step 0
+__device__ __forceinline__ uint32_t score_bin(float x) {
+  const uint32_t w = __float_as_uint(x), a = w & 0x7fffffffu;
+  const bool neg = w > 0x80000000u || a > 0x7f800000u;
+  const int mb = min(max((int)(a >> 18) - kMagBase, 0), 1023);
+  return neg ? (uint32_t)(1023 - mb) : (uint32_t)(1024 + mb);
+}
+// The floats of bin b form the closed interval [lo, hi].  Bin 0 holds -inf
+// (and NaN, which no float comparison admits); callers handle it apart.
+__device__ __forceinline__ void bin_bounds(uint32_t b, float& lo, float& hi) {
+  const int mb = b >= 1024 ? (int)b - 1024 : 1023 - (int)b;
+  const uint32_t a_lo = mb == 0 ? 0u : (uint32_t)(kMagBase + mb) << 18;
+  const uint32_t a_hi = mb == 1023 ? 0x7f800000u : ((uint32_t)(kMagBase + mb + 1) << 18) - 1u;
+  if (b >= 1024) {
+    lo = __uint_as_float(a_lo);
+    hi = __uint_as_float(a_hi);
+  } else {
+    lo = -__uint_as_float(a_hi);
+    hi = mb == 0 ? -__uint_as_float(1u) : -__uint_as_float(a_lo);  // zeros sit in bin 1024
+  }
+}
+
 struct Smem {
   uint32_t hist[kBins];
   uint32_t warp_tot[kWarps];
   uint32_t sel_bin;
   uint32_t sel_above;
-  uint32_t gt_pos;
+  uint32_t n_out;   // positions written so far
+  uint32_t n_cand;  // members of bin b1 seen in pass 2
 };
 
 // Given hist[0..nbins) and the number `need` of elements still to take,
@@ -70,10 +109,23 @@ __device__ void find_bin(Smem& sm, int nbins, uint32_t need) {
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kThreads) topk_kernel(Rows R, int32_t row0, const float* scores,
-                                                        int64_t ld, int k, int32_t* idx,
-                                                        int cache_cap) {
-  extern __shared__ uint32_t cache[];
+// Warp-aggregated append: every lane with `pred` gets a distinct slot of
+// *ctr.  All 32 lanes must call it.
+__device__ __forceinline__ uint32_t warp_append(bool pred, uint32_t* ctr, uint32_t& slot) {
+  const uint32_t mask = __ballot_sync(0xffffffffu, pred);
+  if (!mask) return 0;
+  const int lane = threadIdx.x & 31, leader = __ffs(mask) - 1;
+  uint32_t base = 0;
+  if (lane == leader) base = atomicAdd(ctr, (uint32_t)__popc(mask));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  slot = base + __popc(mask & ((1u << lane) - 1u));
+  return mask;
+}
+
+__global__ void __launch_bounds__(kThreads, 3) topk_kernel(Rows R, int32_t row0, const float* scores,
+                                                           int64_t ld, int k, int32_t* idx) {
+  __shared__ uint32_t ckey[kCand];
+  __shared__ int32_t cpos[kCand];
   __shared__ Smem sm;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int32_t r = row0 + blockIdx.x;
@@ -85,81 +137,188 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(Rows R, int32_t row0, co
     return;
   }
   const float* row = scores + (int64_t)blockIdx.x * ld;
-  const bool cached = n <= cache_cap;
-  auto key_at = [&](int i) -> uint32_t { return cached ? cache[i] : rank_key(__ldg(row + i)); };
+  // Rows start 16-byte aligned when ld is a multiple of 4 (the buffer itself is).
+  const bool vec = (ld & 3) == 0;
 
-  // pass 1: top 11 bits
+  // ------------------------------------------------------------ pass 1
   for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0;
-  if (tid == 0) sm.gt_pos = 0;
+  if (tid == 0) {
+    sm.n_out = 0;
+    sm.n_cand = 0;
+  }
   __syncthreads();
-  for (int i = tid; i < n; i += kThreads) {
-    uint32_t u = rank_key(__ldg(row + i));
-    if (cached) cache[i] = u;
-    atomicAdd(&sm.hist[u >> 21], 1u);
+  const float4* row4 = reinterpret_cast<const float4*>(row);
+  const int n4 = (n + 3) >> 2;  // the last vector may run past n (not past ld)
+  if (vec) {
+#pragma unroll 4
+    for (int v = tid; v < n4; v += kThreads) {
+      const float4 x = __ldg(row4 + v);
+      const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (4 * v + e < n) atomicAdd(&sm.hist[score_bin(xs[e])], 1u);
+    }
+  } else {
+    for (int i = tid; i < n; i += kThreads) atomicAdd(&sm.hist[score_bin(__ldg(row + i))], 1u);
   }
   __syncthreads();
   find_bin(sm, kBins, (uint32_t)k);
   const uint32_t b1 = sm.sel_bin;
-  uint32_t above = sm.sel_above;
+  const uint32_t above1 = sm.sel_above;  // scores in bins above b1
+  const uint32_t in_b1 = sm.hist[b1];
+  const uint32_t need = (uint32_t)k - above1;  // 1 <= need <= in_b1
   __syncthreads();
 
-  // pass 2: middle 11 bits among keys whose top bits are b1
-  for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0;
-  __syncthreads();
-  for (int i = tid; i < n; i += kThreads) {
-    uint32_t u = key_at(i);
-    if ((u >> 21) == b1) atomicAdd(&sm.hist[(u >> 10) & 0x7ffu], 1u);
+  // ------------------------------------------------------------ pass 2
+  // Everything above b1 is selected; the members of b1 become candidates
+  // (when they all fit the buffer).
+  const bool collect = in_b1 <= (uint32_t)kCand;
+  float lo, hi;
+  bin_bounds(b1, lo, hi);
+  if (vec && b1 != 0) {
+    // four scores per thread: above hi -> written out (one atomic per warp
+    // and step), in [lo, hi] -> candidates (rare: per-score appends)
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int base = 0; base < n4; base += kThreads) {  // uniform trip count
+      const int v = base + tid;
+      const float4 x = v < n4 ? __ldg(row4 + v) : make_float4(-INFINITY, -INFINITY, -INFINITY,
+                                                              -INFINITY);
+      const float xs[4] = {x.x, x.y, x.z, x.w};
+      bool gt[4], eq[4];
+      bool any_eq = false;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool ok = 4 * v + e < n;
+        gt[e] = ok && xs[e] > hi;
+        eq[e] = ok && !gt[e] && xs[e] >= lo;
+        any_eq |= eq[e];
+      }
+      uint32_t g[4], tot = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        g[e] = __ballot_sync(0xffffffffu, gt[e]);
+        tot += __popc(g[e]);
+      }
+      if (tot) {
+        uint32_t slot = 0;
+        if (lane == 0) slot = atomicAdd(&sm.n_out, tot);
+        slot = __shfl_sync(0xffffffffu, slot, 0);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (gt[e]) out[slot + __popc(g[e] & lt)] = 4 * v + e;
+          slot += __popc(g[e]);
+        }
+      }
+      if (collect && __any_sync(0xffffffffu, any_eq)) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint32_t slot;
+          if (warp_append(eq[e], &sm.n_cand, slot) && eq[e]) {
+            ckey[slot] = rank_key(xs[e]);
+            cpos[slot] = 4 * v + e;
+          }
+        }
+      }
+    }
+  } else {
+    for (int base = 0; base < n; base += kThreads) {  // uniform trip count
+      const int i = base + tid;
+      const float x = i < n ? __ldg(row + i) : 0.f;
+      const uint32_t b = i < n ? score_bin(x) : 0u;
+      const bool gt = i < n && b > b1, eq = collect && i < n && b == b1;
+      uint32_t slot;
+      if (warp_append(gt, &sm.n_out, slot) && gt) out[slot] = i;
+      if (warp_append(eq, &sm.n_cand, slot) && eq) {
+        ckey[slot] = rank_key(x);
+        cpos[slot] = i;
+      }
+    }
   }
   __syncthreads();
-  find_bin(sm, kBins, (uint32_t)k - above);
-  const uint32_t pre2 = (b1 << 11) | sm.sel_bin;
-  above += sm.sel_above;
-  __syncthreads();
 
-  // pass 3: low 10 bits among keys whose top 22 bits are pre2
-  for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0;
-  __syncthreads();
-  for (int i = tid; i < n; i += kThreads) {
-    uint32_t u = key_at(i);
-    if ((u >> 10) == pre2) atomicAdd(&sm.hist[u & 0x3ffu], 1u);
+  if (collect) {
+    // ---------------------------------------------------------- rank the candidates
+    // rank = candidates with a larger key, or an equal key at a lower
+    // position; the `need` best (rank < need) are taken.
+    const int m = (int)in_b1;
+    for (int base = 0; base < m; base += kThreads) {  // uniform trip count
+      const int j = base + tid;
+      bool take = false;
+      if (j < m) {
+        const uint32_t kj = ckey[j];
+        const int32_t pj = cpos[j];
+        uint32_t rank = 0;
+        for (int l = 0; l < m; ++l) {
+          const uint32_t kl = ckey[l];
+          rank += (kl > kj || (kl == kj && cpos[l] < pj)) ? 1u : 0u;
+        }
+        take = rank < need;
+      }
+      uint32_t slot;
+      if (warp_append(take, &sm.n_out, slot) && take) out[slot] = cpos[j];
+    }
+    return;
   }
-  __syncthreads();
-  find_bin(sm, 1024, (uint32_t)k - above);
-  const uint32_t tau = (pre2 << 10) | sm.sel_bin;
-  const uint32_t c_gt = above + sm.sel_above;  // elements strictly above tau
-  const uint32_t need_eq = (uint32_t)k - c_gt;  // >= 1
-  __syncthreads();
 
-  // pass 4: emit. Elements above tau in any order at [0, c_gt); the first
-  // need_eq elements equal to tau, in position order, at [c_gt, k).
-  uint32_t eq_base = 0;
+  // ------------------------------------------------------------ b1 overflowed the buffer
+  // Three radix levels over the fp32 keys of b1's members, read from the row.
+  auto member_key = [&](int i, uint32_t& u) -> bool {
+    const float x = __ldg(row + i);
+    u = rank_key(x);
+    return score_bin(x) == b1;
+  };
+  uint32_t prefix = 0, c_gt = above1;
+  const int shift[3] = {21, 10, 0};
+  const uint32_t width[3] = {11, 11, 10};
+#pragma unroll
+  for (int lvl = 0; lvl < 3; ++lvl) {
+    for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0;
+    __syncthreads();
+    const int hi = shift[lvl] + (int)width[lvl];  // bits above this level must match prefix
+    for (int i = tid; i < n; i += kThreads) {
+      uint32_t u;
+      if (member_key(i, u) && (hi >= 32 || (u >> hi) == prefix))
+        atomicAdd(&sm.hist[(u >> shift[lvl]) & ((1u << width[lvl]) - 1u)], 1u);
+    }
+    __syncthreads();
+    find_bin(sm, 1 << width[lvl], (uint32_t)k - c_gt);
+    prefix = (prefix << width[lvl]) | sm.sel_bin;
+    c_gt += sm.sel_above;
+    __syncthreads();
+  }
+  const uint32_t tau = prefix;                  // the k-th best key
+  const uint32_t need_eq = (uint32_t)k - c_gt;  // >= 1 keys equal to tau to take
+  const uint32_t n_eq = sm.hist[tau & 0x3ffu];
+  __syncthreads();
+  // b1's members above tau in any order; those equal to tau all go when
+  // exactly need_eq of them exist, else the need_eq lowest positions.
+  const bool all_eq = n_eq == need_eq;
   for (int base = 0; base < n; base += kThreads) {
     const int i = base + tid;
-    const uint32_t u = i < n ? key_at(i) : 0u;
-    const bool gt = i < n && u > tau;
-    const bool eq = i < n && u == tau;
-    const uint32_t gmask = __ballot_sync(0xffffffffu, gt);
-    if (gmask) {
-      uint32_t wbase = 0;
-      if (lane == 0) wbase = atomicAdd(&sm.gt_pos, (uint32_t)__popc(gmask));
-      wbase = __shfl_sync(0xffffffffu, wbase, 0);
-      if (gt) out[wbase + __popc(gmask & ((1u << lane) - 1u))] = i;
+    uint32_t u = 0;
+    const bool take = i < n && member_key(i, u) && (u > tau || (all_eq && u == tau));
+    uint32_t slot;
+    if (warp_append(take, &sm.n_out, slot) && take) out[slot] = i;
+  }
+  if (all_eq) return;
+  __syncthreads();
+  uint32_t eq_base = 0;
+  for (int base = 0; base < n && eq_base < need_eq; base += kThreads) {  // uniform
+    const int i = base + tid;
+    const bool eq = i < n && rank_key(__ldg(row + i)) == tau;
+    const uint32_t emask = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) sm.warp_tot[warp] = (uint32_t)__popc(emask);
+    __syncthreads();
+    uint32_t before = 0, total = 0;
+    for (int w2 = 0; w2 < kWarps; ++w2) {
+      const uint32_t c = sm.warp_tot[w2];
+      if (w2 < warp) before += c;
+      total += c;
     }
-    if (eq_base < need_eq) {  // uniform across the block
-      const uint32_t emask = __ballot_sync(0xffffffffu, eq);
-      if (lane == 0) sm.warp_tot[warp] = (uint32_t)__popc(emask);
-      __syncthreads();
-      uint32_t before = 0, total = 0;
-      for (int w2 = 0; w2 < kWarps; ++w2) {
-        uint32_t c = sm.warp_tot[w2];
-        if (w2 < warp) before += c;
-        total += c;
-      }
-      const uint32_t rank = eq_base + before + __popc(emask & ((1u << lane) - 1u));
-      if (eq && rank < need_eq) out[c_gt + rank] = i;
-      eq_base += total;
-      __syncthreads();
-    }
+    const uint32_t rank = eq_base + before + __popc(emask & ((1u << lane) - 1u));
+    if (eq && rank < need_eq) out[c_gt + rank] = i;
+    eq_base += total;
+    __syncthreads();
   }
 }
 
@@ -168,14 +327,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(Rows R, int32_t row0, co
 dsa_status_t launch_topk(const Rows& R, int32_t row0, int32_t nrows, const float* scores,
                          int64_t ld, int k, int32_t* idx, cudaStream_t st) {
   if (nrows <= 0) return DSA_OK;
-  // Rows up to cache_cap entries are parked in shared memory; longer rows
-  // stream from global memory (L2) on every pass.
-  const int cache_cap = R.max_len < kCacheCap ? R.max_len : kCacheCap;
-  const size_t cache_bytes = (size_t)cache_cap * 4;
-  if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)cache_bytes) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  topk_kernel<<<nrows, kThreads, cache_bytes, st>>>(R, row0, scores, ld, k, idx, cache_cap);
+  topk_kernel<<<nrows, kThreads, 0, st>>>(R, row0, scores, ld, k, idx);
   return launch_status();
 }
 
