@@ -13,10 +13,15 @@
 // with no shuffles.  fp8 scales fold in for free: q_scale (positive) moves
 // into w, k_scale multiplies the finished sum.
 //
-// Warp roles (192 threads):
-//   warp 0     TMA producer: the query block once, then a ring of key tiles
-//   warp 1     TMEM allocator and MMA issuer (one thread)
-//   warps 2-5  epilogue: TMEM -> registers, ReLU, weighted head sum, store
+// Warp roles (576 threads):
+//   warp 0      TMA producer: the query block once, then a ring of key tiles
+//   warp 1      TMEM allocator and MMA issuer (one thread)
+//   warps 2-17  epilogue: TMEM -> registers, ReLU, weighted head sum, store.
+//               Four sets of four warps (one warp per TMEM lane quadrant in
+//               each) take one query of every accumulator each, so four
+//               warps per SM sub-partition hide each other's latencies.  A
+//               score costs per head one max (the ReLU) and half of a packed
+//               two-lane fp32 FMA, into four independent accumulator pairs.
 // Key tiles stream through an NK-stage shared-memory ring; accumulators
 // rotate through NS TMEM slots so the MMA of the next job overlaps the
 // epilogue of the previous one.
@@ -36,8 +41,52 @@ using namespace sm100;
 namespace {
 
 constexpr int kHI = 64, kDI = 128, kTileK = 128;  // heads, dims, keys per tile
-constexpr int kThreads = 192;
+constexpr int kThreads = 576;
+constexpr int kEpiThreads = 512;  // warps 2-17
+constexpr int kEpiSets = kEpiThreads / 128;
 constexpr int kDecodeChunk = 2048;  // keys per CTA in decode
+
+// Two fp32 FMAs in one instruction: {lo, hi} = {x0 * w0, x1 * w1} + acc.
+__device__ __forceinline__ uint64_t fma2(float x0, float x1, float w0, float w1, uint64_t acc) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 x, w;\n\t"
+      "mov.b64 x, {%1, %2};\n\t"
+      "mov.b64 w, {%3, %4};\n\t"
+      "fma.rn.f32x2 %0, x, w, %5;\n\t}"
+      : "=l"(d)
+      : "f"(x0), "f"(x1), "f"(w0), "f"(w1), "l"(acc));
+  return d;
+}
+__device__ __forceinline__ float lo32(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi32(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+
+// 64 consecutive fp32 columns of this warp's 32 TMEM lanes (two loads, one wait).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+        "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr), "r"(taddr + 32)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
 
 template <int DT, int G, int NG, int NK>
 struct Cfg {
@@ -165,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < C::NS; ++i) {
       mbar_init(s_full(i), 1);
-      mbar_init(s_empty(i), 4);
+      mbar_init(s_empty(i), kEpiThreads / 32);  // every epilogue warp
     }
     mbar_init(q_full, 1);
     mbar_init(drain, 1);
@@ -256,9 +305,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int et = tid - 64;           // 0..127
+    const int et = tid - 64;           // 0..511
     const int quad = warp & 3;         // TMEM lane quadrant this warp may read
-    for (int i = et; i < C::QB * kHI; i += 128) {
+    const int set = et >> 7;           // warps 2-5: set 0, 6-9: set 1, ...
+    for (int i = et; i < C::QB * kHI; i += kEpiThreads) {
       const int qi = i / kHI, h = i - qi * kHI;
       const int32_t tq = wk.t0 + qi;
       float v = 0.f;
@@ -269,7 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       wq[i] = v;
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+    // queries of an accumulator this set handles (sets beyond G idle)
+    constexpr int QS = G >= kEpiSets ? G / kEpiSets : 1;
+    const bool active = set < G;
     int job = 0;
     for (int j = 0; j < n_tiles; ++j) {
       const int32_t s = (wk.kt_begin + j) * kTileK + quad * 32 + lane;
@@ -283,26 +336,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        if (active) {
 #pragma unroll 1
-        for (int qq = 0; qq < G; ++qq) {
-          const int qi = g * G + qq;
-          const float* wr = wq + qi * kHI;
-          const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + slot * C::N + qq * kHI;
-          float acc = 0.f;
+          for (int qs = 0; qs < QS; ++qs) {
+            const int qq = set * QS + qs;
+            const int qi = g * G + qq;
+            const float4* wr = reinterpret_cast<const float4*>(wq + qi * kHI);
+            const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + slot * C::N + qq * kHI;
+            uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            float v[32];
-            tmem_ld32(ta + half * 32, v);
+            for (int half = 0; half < 2; ++half) {
+              float v[32];
+              tmem_ld32(ta + 32 * half, v);
 #pragma unroll
-            for (int h = 0; h < 32; ++h) acc = fmaf(wr[half * 32 + h], fmaxf(v[h], 0.f), acc);
-          }
-          const int32_t tq = wk.t0 + qi;
-          if (tq >= wk.qvalid_lo && tq < wk.qvalid_hi && s < R.max_len) {
-            float* o = scores + (int64_t)(wk.qrow0 + qi - row0) * ld;
-            if (s <= tq)
-              o[s] = acc * ks;
-            else if (fill)
-              o[s] = -INFINITY;
+              for (int h4 = 0; h4 < 8; ++h4) {
+                const float4 w4 = wr[8 * half + h4];
+                acc[(2 * h4) & 3] = fma2(fmaxf(v[4 * h4], 0.f), fmaxf(v[4 * h4 + 1], 0.f), w4.x,
+                                         w4.y, acc[(2 * h4) & 3]);
+                acc[(2 * h4 + 1) & 3] = fma2(fmaxf(v[4 * h4 + 2], 0.f), fmaxf(v[4 * h4 + 3], 0.f),
+                                             w4.z, w4.w, acc[(2 * h4 + 1) & 3]);
+              }
+            }
+            const float sum = (lo32(acc[0]) + hi32(acc[0])) + (lo32(acc[1]) + hi32(acc[1])) +
+                              ((lo32(acc[2]) + hi32(acc[2])) + (lo32(acc[3]) + hi32(acc[3])));
+            const int32_t tq = wk.t0 + qi;
+            if (tq >= wk.qvalid_lo && tq < wk.qvalid_hi && s < R.max_len) {
+              float* o = scores + (int64_t)(wk.qrow0 + qi - row0) * ld;
+              if (s <= tq)
+                o[s] = sum * ks;
+              else if (fill)
+                o[s] = -INFINITY;
+            }
           }
         }
         tc_fence_before();
@@ -318,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* o = scores + (int64_t)(wk.qrow0 + qi - row0) * ld;
         const int32_t from = wk.kt_end * kTileK;
         const int32_t to = DECODE ? wk.fill_hi : R.max_len;
-        for (int s = from + et; s < to; s += 128) o[s] = -INFINITY;
+        for (int s = from + et; s < to; s += kEpiThreads) o[s] = -INFINITY;
       }
     }
   }
