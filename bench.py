@@ -306,6 +306,22 @@ def roofline(wl, stage_ms, peaks):
             "launch_ms": round(per_launch_ms, 4)}, shares
 
 
+# --------------------------------------------------------------- ranks
+def max_over_ranks(x, world, device):
+    """The largest of every rank's x (all ranks call it, in the same order)."""
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.item()
+
+
+def job_throughput(units_per_rank, ms_max, world):
+    """Whole-job units/s: every rank processes its own replica of the workload
+    (weak scaling), and the job takes as long as its slowest rank."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
 # --------------------------------------------------------------- oracle runs
 def oracle_rows(wl, rows):
     """Runs the whole oracle path (indexer, top-k, attention) on `rows`."""
@@ -416,20 +432,13 @@ def main():
                                                         not a.no_e2e)
         dec = (dwl, dms, dstage, dlaunch, de2e)
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return t.item()
-
-    ms = max_over_ranks(ms)
-    e2e_ms = max_over_ranks(e2e["ms_per_step"]) if e2e else None
+    ms = max_over_ranks(ms, world, "cuda")
+    e2e_ms = max_over_ranks(e2e["ms_per_step"], world, "cuda") if e2e else None
     if dec:
-        dms = max_over_ranks(dec[1])
-        de2e_ms = max_over_ranks(dec[4]["ms_per_step"]) if dec[4] else None
+        dms = max_over_ranks(dec[1], world, "cuda")
+        de2e_ms = max_over_ranks(dec[4]["ms_per_step"], world, "cuda") if dec[4] else None
     tokens = wl.n_q
-    value = world * tokens / (ms * 1e-3)
+    value = job_throughput(tokens, ms, world)
     roof, shares = roofline(wl, stage_ms, peaks)
     if rank == 0:
         cfg = wl.cfg
@@ -446,7 +455,7 @@ def main():
             "gpu_launches": launches,
         }
         if e2e:
-            line["e2e"] = {"value": round(world * tokens / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+            line["e2e"] = {"value": round(job_throughput(tokens, e2e_ms, world), 1), "unit": "tokens/s",
                            "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                            "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]}
         if clocks:
@@ -455,13 +464,13 @@ def main():
             dwl = dec[0]
             droof, dshares = roofline(dwl, dec[2], peaks)
             line["decode"] = {"workload": DESCR[dwl.cfg.cid],
-                              "value": round(world * dwl.n_q / (dms * 1e-3), 1),
+                              "value": round(job_throughput(dwl.n_q, dms, world), 1),
                               "unit": "tokens/s", "ms_per_step": round(dms, 4),
                               "roofline": droof, "stage_share": dshares,
                               "gpu_launches": dec[3]}
             if dec[4]:
                 line["decode"]["e2e"] = {
-                    "value": round(world * dwl.n_q / (de2e_ms * 1e-3), 1), "unit": "tokens/s",
+                    "value": round(job_throughput(dwl.n_q, de2e_ms, world), 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": dec[4]["h2d_bytes_per_step"],
                     "d2h_bytes_per_step": dec[4]["d2h_bytes_per_step"]}
         if world == 1 and not a.no_cpu_baseline:
