@@ -27,7 +27,7 @@
 //   atoms), two stages of 64 gathered cache rows (nine atoms of 64 dims,
 //   K-major for QK, MN-major for PV), and the tile's probabilities P (bf16,
 //   K-major) for PV.
-// The gather: 192 producer threads fetch the selected rows with 16-byte
+// The gather: 224 producer threads fetch the selected rows with 16-byte
 // cp.async, eight lanes per 128-byte segment, straight into the swizzled
 // layout the MMA reads (an empty slot -1 is zero-filled).  Measured on B200
 // (scattered rows, L2-resident source): cp.async sustains about 16 B/cycle
@@ -35,11 +35,11 @@
 // bounded number of bytes in flight -- while one thread issuing TMA
 // tile::gather4 (4 rows per instruction) manages about 4.
 //
-// Warp roles (480 threads per CTA):
-//   warps 0-5   gather producer (indices -> shared memory, cp.async rows)
-//   warp 6      TMEM allocator and MMA issuer (one thread, issues whichever of
+// Warp roles (512 threads per CTA):
+//   warps 0-6   gather producer (indices -> shared memory, cp.async rows)
+//   warp 7      TMEM allocator and MMA issuer (one thread, issues whichever of
 //               QK(next tile) and PV(oldest tile with P ready) can go)
-//   warps 7-14  softmax, two warpgroups: a thread owns one head (its TMEM
+//   warps 8-15  softmax, two warpgroups: a thread owns one head (its TMEM
 //               lane) and half of each tile's 64 rows.  Online softmax in the
 //               log2 domain with a lazy rescale (the reference max moves only
 //               when a new score exceeds it by more than 2^8); P to shared
@@ -62,11 +62,11 @@ namespace {
 constexpr int kH = 128, kDK = 576, kDV = 512;
 constexpr int kNT = 64;                        // selected rows per tile
 constexpr int kAtoms = kDK / 64;               // 9 swizzle atoms per gathered row
-constexpr int kProducers = 192;                // warps 0-5
-constexpr int kMmaWarp = 6;
-constexpr int kSoftmax0 = 224;                 // first softmax thread (warps 7-14)
+constexpr int kProducers = 224;                // warps 0-6
+constexpr int kMmaWarp = 7;
+constexpr int kSoftmax0 = 256;                 // first softmax thread (warps 8-15)
 constexpr int kSoftmaxThreads = 256;
-constexpr int kThreads = kSoftmax0 + kSoftmaxThreads;  // 480
+constexpr int kThreads = kSoftmax0 + kSoftmaxThreads;  // 512
 constexpr int kAtomBytes = kNT * 128;          // 8192: one 64-dim atom of a tile
 constexpr int kCBytes = kAtoms * kAtomBytes;   // 73728 per stage
 constexpr int kStages = 2;
