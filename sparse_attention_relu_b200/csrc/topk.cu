@@ -122,6 +122,92 @@ __device__ __forceinline__ uint32_t warp_append(bool pred, uint32_t* ctr, uint32
   return mask;
 }
 
+// Writes the `need` best of m candidates (key, position) to dst[0 .. need):
+// rank = candidates with a larger key, or an equal key at a lower position
+// (the tie rule), and candidate j goes to dst[rank] when rank < need.  All
+// threads of the CTA call it.
+__device__ void rank_candidates(const uint32_t* ckey, const int32_t* cpos, int m, uint32_t need,
+                                int32_t* dst) {
+  for (int j = threadIdx.x; j < m; j += kThreads) {
+    const uint32_t kj = ckey[j];
+    const int32_t pj = cpos[j];
+    uint32_t rank = 0;
+    for (int l = 0; l < m; ++l) {
+      const uint32_t kl = ckey[l];
+      rank += (kl > kj || (kl == kj && cpos[l] < pj)) ? 1u : 0u;
+    }
+    if (rank < need) dst[rank] = pj;
+  }
+}
+
+// The members of bin b1 (more than the candidate buffer holds) resolved from
+// the row itself: three radix levels over their fp32 keys find the k-th key
+// tau; members above tau are written after the `above1` scores above b1
+// (sm.n_out counts the written slots), and ties at tau fill the rest from
+// the lowest positions by an ordered pass over the row.  All threads call it.
+__device__ void resolve_by_row(Smem& sm, const float* row, int n, int k, uint32_t b1,
+                               uint32_t above1, int32_t* out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  auto member_key = [&](int i, uint32_t& u) -> bool {
+    const float x = __ldg(row + i);
+    u = rank_key(x);
+    return score_bin(x) == b1;
+  };
+  uint32_t prefix = 0, c_gt = above1;
+  const int shift[3] = {21, 10, 0};
+  const uint32_t width[3] = {11, 11, 10};
+#pragma unroll
+  for (int lvl = 0; lvl < 3; ++lvl) {
+    for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0;
+    __syncthreads();
+    const int hi = shift[lvl] + (int)width[lvl];  // bits above this level must match prefix
+    for (int i = tid; i < n; i += kThreads) {
+      uint32_t u;
+      if (member_key(i, u) && (hi >= 32 || (u >> hi) == prefix))
+        atomicAdd(&sm.hist[(u >> shift[lvl]) & ((1u << width[lvl]) - 1u)], 1u);
+    }
+    __syncthreads();
+    find_bin(sm, 1 << width[lvl], (uint32_t)k - c_gt);
+    prefix = (prefix << width[lvl]) | sm.sel_bin;
+    c_gt += sm.sel_above;
+    __syncthreads();
+  }
+  const uint32_t tau = prefix;                  // the k-th best key
+  const uint32_t need_eq = (uint32_t)k - c_gt;  // >= 1 keys equal to tau to take
+  const uint32_t n_eq = sm.hist[tau & 0x3ffu];
+  __syncthreads();
+  // b1's members above tau in any order; those equal to tau all go when
+  // exactly need_eq of them exist, else the need_eq lowest positions.
+  const bool all_eq = n_eq == need_eq;
+  for (int base = 0; base < n; base += kThreads) {
+    const int i = base + tid;
+    uint32_t u = 0;
+    const bool take = i < n && member_key(i, u) && (u > tau || (all_eq && u == tau));
+    uint32_t slot;
+    if (warp_append(take, &sm.n_out, slot) && take) out[slot] = i;
+  }
+  if (all_eq) return;
+  __syncthreads();
+  uint32_t eq_base = 0;
+  for (int base = 0; base < n && eq_base < need_eq; base += kThreads) {  // uniform
+    const int i = base + tid;
+    const bool eq = i < n && rank_key(__ldg(row + i)) == tau;
+    const uint32_t emask = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) sm.warp_tot[warp] = (uint32_t)__popc(emask);
+    __syncthreads();
+    uint32_t before = 0, total = 0;
+    for (int w2 = 0; w2 < kWarps; ++w2) {
+      const uint32_t c = sm.warp_tot[w2];
+      if (w2 < warp) before += c;
+      total += c;
+    }
+    const uint32_t rank = eq_base + before + __popc(emask & ((1u << lane) - 1u));
+    if (eq && rank < need_eq) out[c_gt + rank] = i;
+    eq_base += total;
+    __syncthreads();
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 3) topk_kernel(Rows R, int32_t row0, const float* scores,
                                                            int64_t ld, int k, int32_t* idx) {
   __shared__ uint32_t ckey[kCand];
@@ -237,88 +323,175 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(Rows R, int32_t row0,
   __syncthreads();
 
   if (collect) {
-    // ---------------------------------------------------------- rank the candidates
-    // rank = candidates with a larger key, or an equal key at a lower
-    // position; the `need` best (rank < need) are taken.
-    const int m = (int)in_b1;
-    for (int base = 0; base < m; base += kThreads) {  // uniform trip count
-      const int j = base + tid;
-      bool take = false;
-      if (j < m) {
-        const uint32_t kj = ckey[j];
-        const int32_t pj = cpos[j];
-        uint32_t rank = 0;
-        for (int l = 0; l < m; ++l) {
-          const uint32_t kl = ckey[l];
-          rank += (kl > kj || (kl == kj && cpos[l] < pj)) ? 1u : 0u;
-        }
-        take = rank < need;
-      }
-      uint32_t slot;
-      if (warp_append(take, &sm.n_out, slot) && take) out[slot] = cpos[j];
-    }
+    rank_candidates(ckey, cpos, (int)in_b1, need, out + above1);
     return;
   }
 
-  // ------------------------------------------------------------ b1 overflowed the buffer
-  // Three radix levels over the fp32 keys of b1's members, read from the row.
-  auto member_key = [&](int i, uint32_t& u) -> bool {
-    const float x = __ldg(row + i);
-    u = rank_key(x);
-    return score_bin(x) == b1;
-  };
-  uint32_t prefix = 0, c_gt = above1;
-  const int shift[3] = {21, 10, 0};
-  const uint32_t width[3] = {11, 11, 10};
+  resolve_by_row(sm, row, n, k, b1, above1, out);
+}
+
+// ---------------------------------------------------------------- split rows
+// Few long rows (decode) leave most SMs idle with one CTA per row, so each
+// row is split over a cluster of kParts CTAs.  Each histograms its slice;
+// the slices' histograms are summed into the leader's (CTA 0) through
+// distributed shared memory (a reduction per non-empty bin), and the leader
+// fixes b1.  Each CTA then filters its slice into local buffers -- scores
+// above b1, and b1's members -- reserves space with one remote atomic on the
+// leader's counters, writes its scores above b1 to the output and its
+// candidates into the leader's buffer.  The leader ranks the candidates (or
+// resolves an overflowing b1 from the row) exactly as the one-CTA kernel.
+constexpr int kParts = 4;
+
+__device__ __forceinline__ uint32_t cl_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cl_map(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(r)
+               : "r"((uint32_t)__cvta_generic_to_shared(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cl_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+__device__ __forceinline__ void cl_red_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t cl_atom_add(uint32_t addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ uint32_t cl_ld(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void cl_st(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads, 2)
+    topk_split_kernel(Rows R, int32_t row0, const float* scores, int64_t ld, int k,
+                      int32_t* idx) {
+  extern __shared__ uint32_t dyn[];
+  uint32_t* ckey = dyn;                                      // [kCand] this slice's candidates
+  int32_t* cpos = reinterpret_cast<int32_t*>(dyn + kCand);   // [kCand]
+  uint32_t* mkey = dyn + 2 * kCand;                          // [kCand] leader: the row's candidates
+  int32_t* mpos = reinterpret_cast<int32_t*>(dyn + 3 * kCand);  // [kCand]
+  __shared__ int32_t gpos[kCand];                            // this slice's scores above b1
+  __shared__ Smem sm;
+  __shared__ uint32_t info[4];  // leader: b1, above1, |b1|; every CTA: its two reservations
+  __shared__ uint32_t local_gt, local_cand;
+  const int tid = threadIdx.x;
+  const uint32_t crank = cl_rank();
+  const int32_t rloc = blockIdx.x / kParts;
+  const RowInfo ri = row_info(R, row0 + rloc);
+  const int n = ri.t + 1;
+  int32_t* out = idx + (int64_t)rloc * k;
+  if (n <= k) {  // the same for every CTA of the cluster
+    if (crank == 0)
+      for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  const float* row = scores + (int64_t)rloc * ld;
+  const bool vec = (ld & 3) == 0;
+  const int chunk = ((n + kParts - 1) / kParts + 3) & ~3;  // slices start 16-byte aligned
+  const int p0 = min(n, (int)crank * chunk), p1 = min(n, p0 + chunk);
+
+  // ------------------------------------------------------------ slice histogram
+  for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0;
+  if (tid == 0) {
+    sm.n_out = 0;  // leader: output slots reserved so far
+    sm.n_cand = 0;  // leader: candidate slots reserved so far
+    local_gt = 0;
+    local_cand = 0;
+  }
+  __syncthreads();
+  if (vec) {
+    const float4* s4 = reinterpret_cast<const float4*>(row + p0);
+    const int m4 = (p1 - p0 + 3) >> 2;
+#pragma unroll 4
+    for (int v = tid; v < m4; v += kThreads) {
+      const float4 x = __ldg(s4 + v);
+      const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-  for (int lvl = 0; lvl < 3; ++lvl) {
-    for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0;
-    __syncthreads();
-    const int hi = shift[lvl] + (int)width[lvl];  // bits above this level must match prefix
-    for (int i = tid; i < n; i += kThreads) {
-      uint32_t u;
-      if (member_key(i, u) && (hi >= 32 || (u >> hi) == prefix))
-        atomicAdd(&sm.hist[(u >> shift[lvl]) & ((1u << width[lvl]) - 1u)], 1u);
+      for (int e = 0; e < 4; ++e)
+        if (p0 + 4 * v + e < p1) atomicAdd(&sm.hist[score_bin(xs[e])], 1u);
     }
-    __syncthreads();
-    find_bin(sm, 1 << width[lvl], (uint32_t)k - c_gt);
-    prefix = (prefix << width[lvl]) | sm.sel_bin;
-    c_gt += sm.sel_above;
-    __syncthreads();
+  } else {
+    for (int i = p0 + tid; i < p1; i += kThreads) atomicAdd(&sm.hist[score_bin(__ldg(row + i))], 1u);
   }
-  const uint32_t tau = prefix;                  // the k-th best key
-  const uint32_t need_eq = (uint32_t)k - c_gt;  // >= 1 keys equal to tau to take
-  const uint32_t n_eq = sm.hist[tau & 0x3ffu];
   __syncthreads();
-  // b1's members above tau in any order; those equal to tau all go when
-  // exactly need_eq of them exist, else the need_eq lowest positions.
-  const bool all_eq = n_eq == need_eq;
-  for (int base = 0; base < n; base += kThreads) {
+  cl_sync();  // every slice histogram complete
+  if (crank != 0)
+    for (int b = tid; b < kBins; b += kThreads) {
+      const uint32_t c = sm.hist[b];
+      if (c) cl_red_add(cl_map(&sm.hist[b], 0), c);
+    }
+  cl_sync();  // the leader holds the row's histogram
+  if (crank == 0) {
+    find_bin(sm, kBins, (uint32_t)k);
+    if (tid == 0) {
+      info[0] = sm.sel_bin;
+      info[1] = sm.sel_above;
+      info[2] = sm.hist[sm.sel_bin];
+    }
+  }
+  cl_sync();
+  if (tid < 3) info[tid] = cl_ld(cl_map(&info[tid], 0));
+  __syncthreads();
+  const uint32_t b1 = info[0], above1 = info[1], in_b1 = info[2];
+  const bool collect = in_b1 <= (uint32_t)kCand;
+  __syncthreads();  // info[0..2] read before the reservations reuse it
+
+  // ------------------------------------------------------------ filter the slice
+  float lo, hi;
+  bin_bounds(b1, lo, hi);
+  for (int base = p0; base < p1; base += kThreads) {  // uniform trip count
     const int i = base + tid;
-    uint32_t u = 0;
-    const bool take = i < n && member_key(i, u) && (u > tau || (all_eq && u == tau));
+    const float x = i < p1 ? __ldg(row + i) : 0.f;
+    bool gt, eq;
+    if (b1 != 0) {
+      gt = i < p1 && x > hi;
+      eq = i < p1 && !gt && x >= lo;
+    } else {  // b1 holds -inf and NaN
+      const uint32_t b = i < p1 ? score_bin(x) : 0u;
+      gt = i < p1 && b > b1;
+      eq = i < p1 && b == b1;
+    }
+    eq = eq && collect;
     uint32_t slot;
-    if (warp_append(take, &sm.n_out, slot) && take) out[slot] = i;
-  }
-  if (all_eq) return;
-  __syncthreads();
-  uint32_t eq_base = 0;
-  for (int base = 0; base < n && eq_base < need_eq; base += kThreads) {  // uniform
-    const int i = base + tid;
-    const bool eq = i < n && rank_key(__ldg(row + i)) == tau;
-    const uint32_t emask = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) sm.warp_tot[warp] = (uint32_t)__popc(emask);
-    __syncthreads();
-    uint32_t before = 0, total = 0;
-    for (int w2 = 0; w2 < kWarps; ++w2) {
-      const uint32_t c = sm.warp_tot[w2];
-      if (w2 < warp) before += c;
-      total += c;
+    if (warp_append(gt, &local_gt, slot) && gt) gpos[slot] = i;  // < above1 < k <= kCand
+    if (warp_append(eq, &local_cand, slot) && eq) {
+      ckey[slot] = rank_key(x);
+      cpos[slot] = i;
     }
-    const uint32_t rank = eq_base + before + __popc(emask & ((1u << lane) - 1u));
-    if (eq && rank < need_eq) out[c_gt + rank] = i;
-    eq_base += total;
-    __syncthreads();
+  }
+  __syncthreads();
+  const uint32_t ngt = local_gt, ncand = local_cand;
+  if (tid == 0) {
+    info[0] = cl_atom_add(cl_map(&sm.n_out, 0), ngt);
+    info[1] = ncand ? cl_atom_add(cl_map(&sm.n_cand, 0), ncand) : 0u;
+  }
+  __syncthreads();
+  const uint32_t base_gt = info[0], base_c = info[1];
+  for (uint32_t j = tid; j < ngt; j += kThreads) out[base_gt + j] = gpos[j];
+  for (uint32_t j = tid; j < ncand; j += kThreads) {
+    cl_st(cl_map(&mkey[base_c + j], 0), ckey[j]);
+    cl_st(cl_map(&mpos[base_c + j], 0), (uint32_t)cpos[j]);
+  }
+  cl_sync();  // every score above b1 written, every candidate with the leader
+
+  if (crank == 0) {
+    if (collect)
+      rank_candidates(mkey, mpos, (int)in_b1, (uint32_t)k - above1, out + above1);
+    else
+      resolve_by_row(sm, row, n, k, b1, above1, out);  // sm.n_out == above1 here
   }
 }
 
@@ -327,6 +500,16 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(Rows R, int32_t row0,
 dsa_status_t launch_topk(const Rows& R, int32_t row0, int32_t nrows, const float* scores,
                          int64_t ld, int k, int32_t* idx, cudaStream_t st) {
   if (nrows <= 0) return DSA_OK;
+  // Few long rows: one cluster of kParts CTAs per row; otherwise one CTA per
+  // row, several per SM.
+  if (k <= kCand && nrows * kParts <= 4 * num_sms() && R.max_len >= 8 * k) {
+    const size_t smem = 4 * kCand * sizeof(uint32_t);  // + static: above the 48 KB default
+    if (cudaFuncSetAttribute(topk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    topk_split_kernel<<<nrows * kParts, kThreads, smem, st>>>(R, row0, scores, ld, k, idx);
+    return launch_status();
+  }
   topk_kernel<<<nrows, kThreads, 0, st>>>(R, row0, scores, ld, k, idx);
   return launch_status();
 }
