@@ -259,6 +259,30 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
     return {"ms_per_step": ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
+KERNEL_SOURCES = {"indexer": "indexer_tc.cu", "topk": "topk.cu", "sparse_mla_attn": "attn_tc.cu"}
+
+
+def measured_traffic(kernel, cid):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+    `kernel` on workload `cid`, from the ncu capture recorded in
+    profiles/dram_traffic.json -- or None when there is none, or when the
+    kernel's source has changed since (the record keeps its SHA-256)."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(f"{kernel}/{cid}")
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "sparse_attention_relu_b200", "csrc", KERNEL_SOURCES[kernel])
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+            return None
+    return rec["bytes_per_launch"]
+
+
 def roofline(wl, stage_ms, peaks):
     """Dominant kernel (largest share of the step) against its roofline."""
     w = algorithmic_work(wl)
@@ -299,7 +323,8 @@ def roofline(wl, stage_ms, peaks):
     names = {0: "indexer", 1: "topk", 2: "sparse_mla_attn", 3: "split_combine"}
     shares = {names[k]: round(v / sum(tot.values()), 4) for k, v in tot.items()}
     return {"kernel": names[kind], "bound": bound, "achieved": round(achieved, 2),
-            "peak": peak, "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
+            "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
+            "traffic": measured_traffic(names[kind], c.cid),
             "peak_source": peaks["source"] + (" (x2 nominal fp8/bf16 ratio)" if
                                              unit == "TFLOP/s" and kind == 0 and
                                              c.idx_dtype == "e4m3" else ""),

@@ -27,8 +27,10 @@
 //   atoms), two stages of 64 gathered cache rows (nine atoms of 64 dims,
 //   K-major for QK, MN-major for PV), and the tile's probabilities P (bf16,
 //   K-major) for PV.
-// The gather: 224 producer threads fetch the selected rows with 16-byte
-// cp.async, eight lanes per 128-byte segment, straight into the swizzled
+// The gather: 224 producer threads fetch the QK-only atoms of each tile and
+// the 256 softmax threads, idle while the tensor cores work on the next
+// tile, fetch this CTA's value atoms, all with 16-byte cp.async, eight lanes
+// per 128-byte segment, straight into the swizzled
 // layout the MMA reads (an empty slot -1 is zero-filled).  Measured on B200
 // (scattered rows, L2-resident source): cp.async sustains about 16 B/cycle
 // per SM from 2 producer warps, 30 from 4 and 40 from 16 -- a warp keeps a
@@ -115,7 +117,8 @@ enum {
   B_SEMPTY = 10,  // scores read (every softmax thread)
   B_PFULL = 11,   // P stored (every softmax thread)
   B_PVDONE = 12,  // PV retired
-  B_DRAIN = 13
+  B_DRAIN = 13,
+  B_IDX = 14      // [2] the tile's indices are in the ring (producers)
 };
 static_assert(B_DRAIN < kNumBars, "barrier count");
 
@@ -235,7 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kStages; ++i) {
       // per producer: an arrive after the index store and a cp.async arrive
       mbar_init(bar(B_AFULL + i), 2 * kProducers);
-      mbar_init(bar(B_VFULL + i), kProducers);  // a cp.async arrive per producer
+      mbar_init(bar(B_VFULL + i), kSoftmaxThreads);  // a cp.async arrive per softmax thread
+      mbar_init(bar(B_IDX + i), kProducers);
       mbar_init(bar(B_AEMPTY + i), 1);
       mbar_init(bar(B_VEMPTY + i), 1);
     }
@@ -255,6 +259,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  // Group V of tile n (this CTA's value columns, 2048 16-byte chunks) is
+  // fetched by the softmax threads, which are otherwise idle while the
+  // tensor cores work on the next tile; thread t issues chunks t + 256 j.
+  // Indices come from the ring the producers fill.
+  const char* const kvrow0 = reinterpret_cast<const char*>(kv + ri.kbase * kDK);
+  auto issue_v = [&](int n) {
+    const int st = n % kStages, ring = n % kIdxRing, t = tid - kSoftmax0;
+#pragma unroll
+    for (int j = 0; j < kChunksV / kSoftmaxThreads; ++j) {
+      const int i = t + kSoftmaxThreads * j;
+      const int ch = i & 7, seg = i >> 3, row = seg >> 2, atom = 4 * half + (seg & 3);
+      const int32_t s = sidx[ring * kNT + row];
+      const char* src = s >= 0 ? kvrow0 + (int64_t)s * (kDK * 2) + atom * 128 + ch * 16
+                               : reinterpret_cast<const char*>(kv);
+      const uint32_t nbytes = s >= 0 ? 16u : 0u;  // 0: zero-fill
+      const uint32_t dst = sb + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128 +
+                           ((uint32_t)(ch ^ (row & 7)) << 4);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                   "r"(nbytes)
+                   : "memory");
+    }
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_VFULL + st))
+                 : "memory");
+  };
+  // Waits until group V of tile n may be fetched: its indices are published
+  // and PV(n-2) released the stage's value atoms.
+  auto v_ready = [&](int n) -> bool {
+    const int st = n % kStages;
+    return mbar_wait(bar(B_IDX + st), (n / kStages) & 1, R.status) &&
+           mbar_wait(bar(B_VEMPTY + st), ((n / kStages) & 1) ^ 1, R.status);
+  };
 
   if (warp < kMmaWarp) {
     // ------------------------------------------------------------ gather producer
@@ -308,24 +344,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) vmask[ring * 2 + warp] = bits;
       }
       mbar_arrive(bar(B_AFULL + st));  // publishes indices and mask to the softmax threads
+      mbar_arrive(bar(B_IDX + st));    // ... and to the threads fetching group V
       asm volatile("bar.sync 2, %0;" ::"n"(kProducers) : "memory");  // producers see the indices
       if (tid < kNT) pre = n + 1 < ntiles ? load_idx(n + 1) : -1;  // overlaps the copies below
 #pragma unroll
       for (int j = 0; j < (kChunksA + kProducers - 1) / kProducers; ++j)
         if (tid + kProducers * j < kChunksA) issue(st, ring, tid + kProducers * j, true);
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_AFULL + st))
-                   : "memory");
-      // group V of the stage is free once PV(n-2) retired
-      ok = mbar_wait(bar(B_VEMPTY + st), par, R.status) && !*abort_flag;
-      if (!bar_and<2, kProducers>(ok)) {
-        *abort_flag = 1;
-        break;
-      }
-#pragma unroll
-      for (int j = 0; j < (kChunksV + kProducers - 1) / kProducers; ++j)
-        if (tid + kProducers * j < kChunksV) issue(st, ring, tid + kProducers * j, false);
-      // arrives on the barrier once this thread's copies (groups A and V) have landed
-      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_VFULL + st))
                    : "memory");
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
@@ -483,6 +508,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_QREADY));
     }
+    // group V of the first two tiles
+    for (int n = 0; n < kStages && n < ntiles; ++n) {
+      if (v_ready(n))
+        issue_v(n);
+      else
+        *abort_flag = 1;
+    }
     // row h of P: this warpgroup's 32 rows are 16-byte chunks 4wg .. 4wg+3
     uint8_t* const prow = smem + OFF_P + h * 128;
     float m2 = -INFINITY, l = 0.f;
@@ -490,10 +522,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int n = 0; ok && n < ntiles; ++n) {
       const int st = n % kStages;
       float s[32];
-      // the tile's validity bits were published with its group A
-      bool w_ok = __all_sync(0xffffffffu,
-                             mbar_wait(bar(B_AFULL + st), (n / kStages) & 1, R.status) &&
-                                 mbar_wait(bar(B_SFULL), n & 1, R.status) && !*abort_flag);
+      // S(n) retired.  The tile's validity bits are already visible: this
+      // thread waited for their publication (B_IDX) before fetching the
+      // tile's group V.  (No wait on B_AFULL here: the producers may already
+      // have refilled the stage's group A for tile n+2, two phases on, which
+      // a parity wait would never see complete.)
+      bool w_ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), n & 1, R.status) && !*abort_flag);
       if (w_ok) {
         tc_fence_after();
         tmem_ld32(tmem + lane_off + TM_S + 32 * wg, s);
@@ -558,8 +592,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();          // P stores before the PV MMA reads them
       tc_fence_before();           // a rescale's TMEM stores before the PV MMA
       mbar_arrive(bar(B_PFULL));
+      // group V of tile n+2 goes into this stage once PV(n) has read it
+      if (n + kStages < ntiles) {
+        if (v_ready(n + kStages))
+          issue_v(n + kStages);
+        else
+          *abort_flag = 1;
+      }
     }
     if (!ok) *abort_flag = 1;
+    asm volatile("cp.async.wait_all;" ::: "memory");  // no group-V copy outlives the CTA
     // combine the two warpgroups' denominators (the first barrier retires the
     // last tile's reads of the half maxima)
     asm volatile("bar.sync 1, 256;" ::: "memory");

@@ -452,24 +452,51 @@ __global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads, 2)
   // ------------------------------------------------------------ filter the slice
   float lo, hi;
   bin_bounds(b1, lo, hi);
-  for (int base = p0; base < p1; base += kThreads) {  // uniform trip count
-    const int i = base + tid;
-    const float x = i < p1 ? __ldg(row + i) : 0.f;
-    bool gt, eq;
+  // score i of the slice is above b1 / a member of b1 (the -inf bin 0 holds
+  // NaN too, which no float comparison admits: compare bins there)
+  auto classify = [&](float x, bool valid, bool& gt, bool& eq) {
     if (b1 != 0) {
-      gt = i < p1 && x > hi;
-      eq = i < p1 && !gt && x >= lo;
-    } else {  // b1 holds -inf and NaN
-      const uint32_t b = i < p1 ? score_bin(x) : 0u;
-      gt = i < p1 && b > b1;
-      eq = i < p1 && b == b1;
+      gt = valid && x > hi;
+      eq = valid && !gt && x >= lo;
+    } else {
+      const uint32_t b = valid ? score_bin(x) : 0u;
+      gt = valid && b > b1;
+      eq = valid && b == b1;
     }
     eq = eq && collect;
-    uint32_t slot;
-    if (warp_append(gt, &local_gt, slot) && gt) gpos[slot] = i;  // < above1 < k <= kCand
-    if (warp_append(eq, &local_cand, slot) && eq) {
-      ckey[slot] = rank_key(x);
-      cpos[slot] = i;
+  };
+  if (vec) {
+    const float4* s4 = reinterpret_cast<const float4*>(row + p0);
+    const int m4 = (p1 - p0 + 3) >> 2;
+    for (int base = 0; base < m4; base += kThreads) {  // uniform trip count
+      const int v = base + tid;
+      const float4 x = v < m4 ? __ldg(s4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = p0 + 4 * v + e;
+        bool gt, eq;
+        classify(xs[e], v < m4 && i < p1, gt, eq);
+        uint32_t slot;
+        if (warp_append(gt, &local_gt, slot) && gt) gpos[slot] = i;  // < above1 < k <= kCand
+        if (warp_append(eq, &local_cand, slot) && eq) {
+          ckey[slot] = rank_key(xs[e]);
+          cpos[slot] = i;
+        }
+      }
+    }
+  } else {
+    for (int base = p0; base < p1; base += kThreads) {  // uniform trip count
+      const int i = base + tid;
+      const float x = i < p1 ? __ldg(row + i) : 0.f;
+      bool gt, eq;
+      classify(x, i < p1, gt, eq);
+      uint32_t slot;
+      if (warp_append(gt, &local_gt, slot) && gt) gpos[slot] = i;
+      if (warp_append(eq, &local_cand, slot) && eq) {
+        ckey[slot] = rank_key(x);
+        cpos[slot] = i;
+      }
     }
   }
   __syncthreads();
