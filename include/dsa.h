@@ -152,15 +152,13 @@ size_t dsa_sparse_mla_attn_workspace_size(const dsa_layout_t* layout, int32_t k,
  * capture mode, code inside a framework whose memory pool owns the whole
  * device, or plug-ins that are handed tensors but no allocator.  This call
  * takes the same arguments as dsa_sparse_mla_attn minus the workspace: the
- * decode split partials go to a fixed 36 MiB array that the library owns
+ * decode split partials go to a fixed 20 MiB array that the library owns
  * on every GPU where it is loaded, held until the process exits.
- *  - Capacity: a call whose split plan needs more than 36 MiB of partials
- *    (128 heads x 513 floats per (query row, split) pair, so at most 143
- *    pairs) returns DSA_ERR_WORKSPACE without launching anything.  Batches
- *    of 74 query rows or more are not split and need no partials; below
- *    that, with k <= 2048, only 72 and 73 rows (144 and 146 pairs) exceed
- *    the array.  Shapes that do not run on the tensor cores need no
- *    scratch and are never refused for size.
+ *  - Capacity: 79 (query row, split) blocks of 128 heads x 513 floats.  The
+ *    split plan of both attention entry points keeps every CTA pair in one
+ *    wave (74 pairs on a 148-SM B200) and never uses more blocks than that,
+ *    so no call is refused for size.  DSA_ERR_WORKSPACE here would mean a
+ *    plan beyond the array, which the planner does not produce.
  *  - Nothing needs zeroing: every call writes each partial it later reads.
  *  - The array is shared by all calls on a device and keeps the last call's
  *    contents: calls whose executions overlap on the GPU (different streams,

@@ -191,17 +191,37 @@ struct Split {
   int nsplit, tiles_per_split;
 };
 
-// Decode rows are few: split each row's tiles so that the CTA pairs cover
-// the 148 SMs (two CTAs per pair, one CTA per SM).
-__host__ __device__ inline Split plan_split(int32_t nrows, int k) {
-  const int tiles = (k + kNT - 1) / kNT;
-  int want = nrows >= 74 ? 1 : (74 + nrows - 1) / nrows;
-  if (want > tiles) want = tiles;
-  if (want < 1) want = 1;
-  Split s;
-  s.tiles_per_split = (tiles + want - 1) / want;
-  s.nsplit = (tiles + s.tiles_per_split - 1) / s.tiles_per_split;
-  return s;
+// Fixed scratch for callers that cannot allocate device memory (see
+// launch_attn_tc_static): the split partials of one call, 20 MiB, room for
+// 79 (query row, split) blocks of 128 x 513 floats.
+constexpr size_t kPartialBytes = size_t(kH) * (kDV + 1) * sizeof(float);
+constexpr size_t kStaticScratchBytes = size_t(20) << 20;
+constexpr int kScratchPairs = int((kStaticScratchBytes - 256) / kPartialBytes);
+static __device__ __align__(256) float g_attn_scratch[kStaticScratchBytes / sizeof(float)];
+
+// Decode rows are few: split each row's tiles over several CTA pairs (two
+// CTAs per pair, one CTA per SM).  Only splits that keep every pair in ONE
+// wave are taken: a second wave costs a whole split's tiles for the pairs
+// that spill into it.  Among those, the estimate is tiles per split plus the
+// merge (each (row, split) block's 256 KiB of fp32 partials go out to memory
+// and back, about 1/48 of a gathered tile's time).  The pair count is capped
+// by the fixed scratch, so both attention entry points plan alike.
+inline Split plan_split(int32_t nrows, int k) {
+  const int tiles = k > 0 ? (k + kNT - 1) / kNT : 1;
+  int pairs = num_sms() / 2;
+  if (pairs > kScratchPairs) pairs = kScratchPairs;
+  Split best{1, tiles};
+  int64_t best_cost = int64_t(tiles) * 48;
+  for (int want = 2; want <= tiles && (int64_t)nrows * want <= pairs; ++want) {
+    const int tps = (tiles + want - 1) / want, ns = (tiles + tps - 1) / tps;
+    if (ns != want) continue;  // same plan as a smaller split
+    const int64_t cost = int64_t(tps) * 48 + (int64_t)nrows * ns;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = Split{ns, tps};
+    }
+  }
+  return best;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -695,12 +715,6 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(int32_t row0, int nsp
   *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
   if (lse && threadIdx.x == 0) lse[(int64_t)r * kH + h] = den > 0.f ? mx + logf(den) : -INFINITY;
 }
-
-// Fixed scratch for callers that cannot allocate device memory (see
-// launch_attn_tc_static): the split partials of one call, 36 MiB (143
-// (query row, split) blocks of 128 x 513 floats).
-constexpr size_t kStaticScratchBytes = size_t(36) << 20;
-static __device__ __align__(256) float g_attn_scratch[kStaticScratchBytes / sizeof(float)];
 
 }  // namespace
 

@@ -47,15 +47,21 @@ def test_noalloc_matches_workspace_call_twice(lens, k):
         _compare(out, lse, ref_out, ref_lse)
 
 
-def test_noalloc_rejects_calls_beyond_its_scratch():
-    """73 decode rows at k = 2048 split in two: 146 partial blocks, more than
-    the 143 the fixed scratch holds -> DSA_ERR_WORKSPACE, nothing launched."""
-    cfg = workloads.custom("decode", [64] * 73, idx_dtype="bf16", k=2048, seed=3)
+@pytest.mark.parametrize("nrows", [37, 64])
+def test_noalloc_largest_split_and_no_split(nrows):
+    """37 rows at k = 2048 split in two: 74 (row, split) blocks, one per CTA
+    pair on 148 SMs, the most any plan uses.  64 rows run unsplit in one
+    wave and need no scratch.  Both match the workspace entry point."""
+    cfg = workloads.custom("decode", [2600 + 40 * i for i in range(nrows)], idx_dtype="bf16",
+                           k=2048, seed=3)
     dev = Dev(workloads.generate(cfg))
-    idx = torch.full((73, 2048), -1, dtype=torch.int32, device="cuda")
-    out = torch.zeros(73, 128, 512, dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(dsa.DSAError) as e:
-        dsa.dsa_sparse_mla_attn_noalloc(dev.layout, dev.d.q, dev.d.kv, idx, 2048, 512,
-                                        cfg.sm_scale, out)
-    assert e.value.status == dsa.DSA_ERR_WORKSPACE
-    assert torch.count_nonzero(out).item() == 0
+    d = dev.d
+    idx = dev.topk(dev.scores())
+    ref_out, ref_lse = dev.attn(idx)
+    out = torch.full_like(ref_out, float("nan"))
+    lse = torch.full_like(ref_lse, float("nan"))
+    dsa.dsa_sparse_mla_attn_noalloc(dev.layout, d.q, d.kv, idx, 2048, cfg.D_V, cfg.sm_scale, out,
+                                    lse)
+    torch.cuda.synchronize()
+    assert dsa.dsa_device_status() == dsa.DSA_OK
+    _compare(out, lse, ref_out, ref_lse)
