@@ -28,7 +28,7 @@
 //
 // Work: prefill -- a CTA owns NG*G consecutive queries of one sequence and
 // every key tile up to the last query (blocks launched heaviest first);
-// decode -- a CTA owns the single query of a sequence and a chunk of KCH keys.
+// decode -- a persistent kernel of its own (indexer_decode_kernel, below).
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
@@ -44,7 +44,6 @@ constexpr int kHI = 64, kDI = 128, kTileK = 128;  // heads, dims, keys per tile
 constexpr int kThreads = 576;
 constexpr int kEpiThreads = 512;  // warps 2-17
 constexpr int kEpiSets = kEpiThreads / 128;
-constexpr int kDecodeChunk = 2048;  // keys per CTA in decode
 
 // Two fp32 FMAs in one instruction: {lo, hi} = {x0 * w0, x1 * w1} + acc.
 __device__ __forceinline__ uint64_t fma2(float x0, float x1, float w0, float w1, uint64_t acc) {
@@ -59,34 +58,6 @@ __device__ __forceinline__ uint64_t fma2(float x0, float x1, float w0, float w1,
 }
 __device__ __forceinline__ float lo32(uint64_t v) { return __uint_as_float((uint32_t)v); }
 __device__ __forceinline__ float hi32(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
-
-// 64 consecutive fp32 columns of this warp's 32 TMEM lanes (two loads, one wait).
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  uint32_t r[64];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
-        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
-        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
-        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
-        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
-        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
-        "=r"(r[62]), "=r"(r[63])
-      : "r"(taddr), "r"(taddr + 32)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 template <int DT, int G, int NG, int NK>
 struct Cfg {
@@ -122,7 +93,6 @@ struct Work {
   int32_t qrow0;      // global query row of query 0 of the block
   int32_t kt_begin, kt_end;  // key tiles
   int32_t qvalid_lo, qvalid_hi;  // valid query positions [lo, hi) (local)
-  int32_t fill_lo, fill_hi;      // decode: key range this CTA owns (for -inf fill)
 };
 
 template <int QB>
@@ -152,28 +122,7 @@ __device__ Work plan_prefill(const Rows& R, int32_t row0, int32_t nrows) {
   return w;
 }
 
-__device__ Work plan_decode(const Rows& R, int32_t row0) {
-  Work w{};
-  const int32_t r = row0 + blockIdx.y;
-  const RowInfo ri = row_info(R, r);
-  const int32_t c0 = blockIdx.x * kDecodeChunk;
-  w.fill_lo = c0;
-  w.fill_hi = min(c0 + kDecodeChunk, R.max_len);
-  w.len = ri.len;
-  w.qrow0 = r;
-  if (ri.t < 0 || c0 > ri.t) return w;  // nothing to score (fill only)
-  w.valid = 1;
-  w.kbase = ri.kbase;
-  w.t0 = ri.t;
-  w.nq = 1;
-  w.qvalid_lo = ri.t;
-  w.qvalid_hi = ri.t + 1;
-  w.kt_begin = c0 / kTileK;
-  w.kt_end = (min(c0 + kDecodeChunk, ri.t + 1) + kTileK - 1) / kTileK;
-  return w;
-}
-
-template <int DT, int G, int NG, int NK, bool DECODE>
+template <int DT, int G, int NG, int NK>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ CUtensorMap kmap, Rows R, int32_t row0,
@@ -197,15 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const Work wk = DECODE ? plan_decode(R, row0) : plan_prefill<C::QB>(R, row0, nrows);
-
-  if (!wk.valid) {
-    if (DECODE && fill && wk.fill_lo < wk.fill_hi) {  // a chunk past the end of the sequence
-      float* o = scores + (int64_t)blockIdx.y * ld;
-      for (int s = wk.fill_lo + tid; s < wk.fill_hi; s += kThreads) o[s] = -INFINITY;
-    }
-    return;
-  }
+  const Work wk = plan_prefill<C::QB>(R, row0, nrows);
+  if (!wk.valid) return;
 
   if (tid == 0) {
     for (int i = 0; i < NK; ++i) {
@@ -320,23 +262,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       wq[i] = v;
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
-    // queries of an accumulator this set handles (sets beyond G idle)
-    constexpr int QS = G >= kEpiSets ? G / kEpiSets : 1;
-    const bool active = set < G;
+    // queries of each accumulator this set handles
+    static_assert(G % kEpiSets == 0, "every epilogue set takes a share of each accumulator");
+    constexpr int QS = G / kEpiSets;
+    // the key scale of this thread's key, loaded one tile ahead
+    auto key_scale = [&](int j) {
+      const int32_t s = (wk.kt_begin + j) * kTileK + quad * 32 + lane;
+      return (DT == DSA_E4M3 && k_scale && j < n_tiles && s < wk.len) ? __ldg(k_scale + wk.kbase + s)
+                                                                      : 1.f;
+    };
+    float ks_next = key_scale(0);
     int job = 0;
     for (int j = 0; j < n_tiles; ++j) {
       const int32_t s = (wk.kt_begin + j) * kTileK + quad * 32 + lane;
-      float ks = 1.f;
-      if (DT == DSA_E4M3 && k_scale && s < wk.len) ks = __ldg(k_scale + wk.kbase + s);
+      const float ks = ks_next;
+      ks_next = key_scale(j + 1);
       for (int g = 0; g < NG; ++g, ++job) {
         const int slot = job % C::NS;
-        if (!mbar_wait(s_full(slot), (job / C::NS) & 1, R.status) || *abort_flag) {
+        // warp-uniform: the tcgen05 loads below need the whole warp
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(s_full(slot), (job / C::NS) & 1, R.status) && !*abort_flag)) {
           *abort_flag = 1;
           j = n_tiles;
           break;
         }
         tc_fence_after();
-        if (active) {
+        {
 #pragma unroll 1
           for (int qs = 0; qs < QS; ++qs) {
             const int qq = set * QS + qs;
@@ -381,10 +332,375 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (qi >= wk.nq || tq < wk.qvalid_lo || tq >= wk.qvalid_hi) continue;
         float* o = scores + (int64_t)(wk.qrow0 + qi - row0) * ld;
         const int32_t from = wk.kt_end * kTileK;
-        const int32_t to = DECODE ? wk.fill_hi : R.max_len;
-        for (int s = from + et; s < to; s += kEpiThreads) o[s] = -INFINITY;
+        for (int s = from + et; s < R.max_len; s += kEpiThreads) o[s] = -INFINITY;
       }
     }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TCOLS);
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// Decode: one query per sequence against its whole cache.  A persistent grid
+// (one CTA per SM) cuts the concatenated key tiles of all rows into equal
+// contiguous ranges, one per CTA; a range may cross row boundaries, and the
+// key stream keeps flowing across them (the query block and head weights of
+// the next row load into the other of two buffers while the current row is
+// scored).  Equal ranges keep every SM streaming keys until the end, where a
+// grid of per-row chunks paid a prologue and a pipeline ramp per chunk and
+// left the last wave ragged.
+template <int DT, int NK>
+struct DecCfg {
+  using C = Cfg<DT, 1, 1, NK>;
+  static constexpr int OFF_Q = 0;                         // [2][64 x ROWB] query blocks
+  static constexpr int OFF_K = 2 * C::QBYTES;             // [NK][128 x ROWB] key ring
+  static constexpr int OFF_W = OFF_K + NK * C::KBYTES;    // [2][64] head weights
+  static constexpr int OFF_SCAN = OFF_W + 2 * kHI * 4;    // block-scan scratch
+  static constexpr int OFF_BAR = OFF_SCAN + 32 * 8 + 32;
+  // k_full/k_empty [NK], s_full/s_empty [NS], q_full/q_empty [2], drain
+  static constexpr int NBAR = 2 * NK + 2 * C::NS + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 32 + 1024;
+  static_assert(C::QBYTES % 1024 == 0 && C::KBYTES % 1024 == 0, "1024-byte operand alignment");
+  static_assert(C::NS % kEpiSets == 0, "a TMEM slot always belongs to the same epilogue set");
+};
+
+// Key tiles of decode row r (0 when the row has no candidates).
+__device__ __forceinline__ int32_t dec_row_tiles(const Rows& R, int32_t r) {
+  const RowInfo ri = row_info(R, r);
+  return ri.t < 0 ? 0 : (ri.t + kTileK) / kTileK;
+}
+
+// Inclusive sum over the block of one value per thread (kThreads threads);
+// `total` receives the block's sum.  Uses 18 int64 words of `scr`.
+__device__ __forceinline__ int64_t block_incl_scan(int64_t v, int64_t* scr, int64_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) scr[warp] = v;
+  __syncthreads();
+  int64_t before = 0, all = 0;
+  for (int i = 0; i < kThreads / 32; ++i) {
+    const int64_t s = scr[i];
+    if (i < warp) before += s;
+    all += s;
+  }
+  __syncthreads();
+  total = all;
+  return v + before;
+}
+
+// One CTA's walk over its tile range: local row r, key tiles [kb, ke) of it,
+// and the tiles of the range that come after this segment.
+struct SegWalk {
+  int32_t r, kb, ke;
+  int64_t left;
+};
+
+__device__ __forceinline__ SegWalk seg_first(const Rows& R, int32_t row0, int32_t r, int32_t off,
+                                             int64_t n) {
+  SegWalk s;
+  s.r = r;
+  s.kb = off;
+  const int64_t take = min((int64_t)(dec_row_tiles(R, row0 + r) - off), n);
+  s.ke = off + (int32_t)take;
+  s.left = n - take;
+  return s;
+}
+
+__device__ __forceinline__ bool seg_next(const Rows& R, int32_t row0, int32_t nrows, SegWalk& s) {
+  while (s.left > 0 && ++s.r < nrows) {
+    const int32_t nt = dec_row_tiles(R, row0 + s.r);
+    if (nt == 0) continue;
+    const int64_t take = min((int64_t)nt, s.left);
+    s.kb = 0;
+    s.ke = (int32_t)take;
+    s.left -= take;
+    return true;
+  }
+  return false;
+}
+
+template <int DT, int NK>
+__global__ void __launch_bounds__(kThreads, 1)
+    indexer_decode_kernel(const __grid_constant__ CUtensorMap qmap,
+                          const __grid_constant__ CUtensorMap kmap, Rows R, int32_t row0,
+                          int32_t nrows, const float* __restrict__ w,
+                          const float* __restrict__ q_scale, const float* __restrict__ k_scale,
+                          float* __restrict__ scores, int64_t ld, int fill) {
+  using D = DecCfg<DT, NK>;
+  using C = typename D::C;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* wq = reinterpret_cast<float*>(smem + D::OFF_W);
+  int64_t* scr = reinterpret_cast<int64_t*>(smem + D::OFF_SCAN);
+  const uint32_t bar0 = sbase + D::OFF_BAR;
+  auto k_full = [&](int i) { return bar0 + 8u * i; };
+  auto k_empty = [&](int i) { return bar0 + 8u * (NK + i); };
+  auto s_full = [&](int i) { return bar0 + 8u * (2 * NK + i); };
+  auto s_empty = [&](int i) { return bar0 + 8u * (2 * NK + C::NS + i); };
+  auto q_full = [&](int b) { return bar0 + 8u * (2 * NK + 2 * C::NS + b); };
+  auto q_empty = [&](int b) { return bar0 + 8u * (2 * NK + 2 * C::NS + 2 + b); };
+  const uint32_t drain = bar0 + 8u * (2 * NK + 2 * C::NS + 4);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + D::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + D::OFF_MISC + 4);
+  volatile int32_t* s_first = reinterpret_cast<volatile int32_t*>(smem + D::OFF_MISC + 8);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t G = gridDim.x;
+
+  // -inf past the last tile of each row (unit call only); row r's tail is
+  // written by CTA r mod G, its tiles by whichever CTA scores them
+  if (fill) {
+    for (int64_t r = blockIdx.x; r < nrows; r += G) {
+      const int32_t from = min(dec_row_tiles(R, row0 + (int32_t)r) * kTileK, R.max_len);
+      float* o = scores + r * ld;
+      for (int32_t s = from + tid; s < R.max_len; s += kThreads) o[s] = -INFINITY;
+    }
+  }
+
+  // ---- this CTA's share of the concatenated key tiles: [T0, T1)
+  int64_t total = 0;
+  for (int32_t r0 = 0; r0 < nrows; r0 += kThreads) {
+    const int32_t r = r0 + tid;
+    int64_t blk;
+    block_incl_scan(r < nrows ? dec_row_tiles(R, row0 + r) : 0, scr, blk);
+    total += blk;
+  }
+  const int64_t T0 = total * blockIdx.x / G, T1 = total * (blockIdx.x + 1) / G;
+  if (T0 >= T1) return;
+  if (tid == 0) s_first[0] = -1;
+  int64_t base = 0;
+  for (int32_t r0 = 0; r0 < nrows; r0 += kThreads) {
+    const int32_t r = r0 + tid;
+    const int32_t n = r < nrows ? dec_row_tiles(R, row0 + r) : 0;
+    int64_t blk;
+    const int64_t excl = base + block_incl_scan(n, scr, blk) - n;
+    if (n > 0 && excl <= T0 && T0 < excl + n) {
+      s_first[0] = r;
+      s_first[1] = (int32_t)(T0 - excl);
+    }
+    base += blk;
+  }
+  __syncthreads();
+  const int32_t first_row = s_first[0], first_off = s_first[1];
+  if (first_row < 0) return;  // offsets changed under us; nothing sensible to do
+  const SegWalk start = seg_first(R, row0, first_row, first_off, T1 - T0);
+
+  if (tid == 0) {
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(k_full(i), 1);
+      mbar_init(k_empty(i), 1);
+    }
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(s_full(i), 1);
+      mbar_init(s_empty(i), 4);  // the four warps of the set that owns the slot
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(q_full(b), 1);
+      mbar_init(q_empty(b), 1 + kEpiThreads / 32);  // MMA commit + every epilogue warp
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + D::OFF_MISC, C::TCOLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    // The whole warp stages the head weights of each row; lane 0 issues
+    // the TMA loads of the query block and the key tiles.
+    if (lane == 0) {
+      tma_prefetch(&qmap);
+      tma_prefetch(&kmap);
+    }
+    SegWalk sg = start;
+    int si = 0, q_issued = 0;
+    int64_t gt = 0, issued = 0;
+    bool ok = true;
+    do {
+      const int qb = si & 1;
+      // buffer qb is free once the MMAs and the epilogue of segment si - 2 are done
+      if (si >= 2) {
+        int free_ok = 1;
+        if (lane == 0)
+          free_ok = mbar_wait(q_empty(qb), ((si - 2) >> 1) & 1, R.status) && !*abort_flag;
+        if (!__shfl_sync(0xffffffffu, free_ok, 0)) {
+          ok = false;
+          break;
+        }
+      }
+      const int64_t qr = (int64_t)row0 + sg.r;  // global query row
+      for (int h = lane; h < kHI; h += 32) {
+        float v = __ldg(w + qr * kHI + h);
+        if (q_scale) v *= __ldg(q_scale + qr * kHI + h);
+        wq[qb * kHI + h] = v;
+      }
+      __syncwarp();
+      int lane_ok = 1;
+      if (lane == 0) {
+        const RowInfo ri = row_info(R, (int32_t)qr);
+        mbar_expect_tx(q_full(qb), C::QBYTES);
+        for (int kc = 0; kc < C::KC; ++kc)
+          tma_load_2d(sbase + D::OFF_Q + qb * C::QBYTES + kc * C::N * 128, &qmap,
+                      kc * (128 / C::ESZ), (int32_t)qr * kHI, q_full(qb));
+        ++q_issued;
+        for (int j = sg.kb; j < sg.ke; ++j, ++gt) {
+          const int st = (int)(gt % NK);
+          if (!mbar_wait(k_empty(st), (int)((gt / NK) & 1) ^ 1, R.status) || *abort_flag) {
+            lane_ok = 0;
+            break;
+          }
+          mbar_expect_tx(k_full(st), C::KBYTES);
+          const int32_t krow = (int32_t)(ri.kbase + (int64_t)j * kTileK);
+          for (int kc = 0; kc < C::KC; ++kc)
+            tma_load_2d(sbase + D::OFF_K + st * C::KBYTES + kc * kTileK * 128, &kmap,
+                        kc * (128 / C::ESZ), krow, k_full(st));
+          ++issued;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, lane_ok, 0) != 0;
+      ++si;
+    } while (ok && seg_next(R, row0, nrows, sg));
+    if (!ok) *abort_flag = 1;
+    if (lane == 0) {
+      // leave no copy in flight behind us
+      for (int64_t j = max((int64_t)0, issued - NK); j < issued; ++j)
+        mbar_wait(k_full((int)(j % NK)), (int)((j / NK) & 1), R.status);
+      for (int s2 = max(0, q_issued - 2); s2 < q_issued; ++s2)
+        mbar_wait(q_full(s2 & 1), (s2 >> 1) & 1, R.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      SegWalk sg = start;
+      int si = 0;
+      int64_t gt = 0;
+      bool ok = true;
+      do {
+        const int qb = si & 1;
+        if (!mbar_wait(q_full(qb), (si >> 1) & 1, R.status) || *abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t b_base = sbase + D::OFF_Q + qb * C::QBYTES;
+        for (int j = sg.kb; j < sg.ke; ++j, ++gt) {
+          const int st = (int)(gt % NK), slot = (int)(gt % C::NS);
+          if (!mbar_wait(k_full(st), (int)((gt / NK) & 1), R.status) ||
+              !mbar_wait(s_empty(slot), (int)((gt / C::NS) & 1) ^ 1, R.status) || *abort_flag) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = sbase + D::OFF_K + st * C::KBYTES;
+          const uint32_t d = tmem + slot * C::N;
+#pragma unroll
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const int kc = kk / 4, sub = (kk % 4) * 32;
+            const uint64_t da = desc_sw128(a_base + kc * kTileK * 128 + sub, 1024);
+            const uint64_t db = desc_sw128(b_base + kc * C::N * 128 + sub, 1024);
+            if constexpr (DT == DSA_BF16)
+              mma_bf16(d, da, db, C::IDESC, kk > 0 ? 1u : 0u);
+            else
+              mma_e4m3(d, da, db, C::IDESC, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(s_full(slot));
+          mma_commit(k_empty(st));
+        }
+        if (!ok) break;
+        mma_commit(q_empty(qb));
+        ++si;
+      } while (seg_next(R, row0, nrows, sg));
+      if (!ok) {
+        *abort_flag = 1;
+        mma_commit(drain);
+        mbar_wait(drain, 0, R.status);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // Set `set` (four warps, one per TMEM lane quadrant) takes every fourth
+    // accumulator: with a single query per accumulator this keeps all
+    // sixteen warps busy.
+    const int et = tid - 64, quad = warp & 3, set = et >> 7;
+    SegWalk sg = start;
+    int si = 0;
+    int64_t gt = 0;
+    bool ok = true;
+    do {
+      const int qb = si & 1;
+      // warp-uniform outcome of each wait: the tcgen05 loads below need the
+      // whole warp, so a lane that gave up takes the others with it
+      if (!__all_sync(0xffffffffu, mbar_wait(q_full(qb), (si >> 1) & 1, R.status) && !*abort_flag)) {
+        ok = false;
+        break;
+      }
+      const RowInfo ri = row_info(R, row0 + sg.r);
+      const float4* wr = reinterpret_cast<const float4*>(wq + qb * kHI);
+      float* o = scores + (int64_t)sg.r * ld;
+      for (int j = sg.kb; j < sg.ke; ++j, ++gt) {
+        if ((int)(gt % kEpiSets) != set) continue;
+        const int slot = (int)(gt % C::NS);
+        const int32_t s = j * kTileK + quad * 32 + lane;
+        float ks = 1.f;
+        if (DT == DSA_E4M3 && k_scale && s <= ri.t) ks = __ldg(k_scale + ri.kbase + s);
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(s_full(slot), (int)((gt / C::NS) & 1), R.status) && !*abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + slot * C::N;
+        uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float v[32];
+          tmem_ld32(ta + 32 * half, v);
+#pragma unroll
+          for (int h4 = 0; h4 < 8; ++h4) {
+            const float4 w4 = wr[8 * half + h4];
+            acc[(2 * h4) & 3] = fma2(fmaxf(v[4 * h4], 0.f), fmaxf(v[4 * h4 + 1], 0.f), w4.x, w4.y,
+                                     acc[(2 * h4) & 3]);
+            acc[(2 * h4 + 1) & 3] = fma2(fmaxf(v[4 * h4 + 2], 0.f), fmaxf(v[4 * h4 + 3], 0.f),
+                                         w4.z, w4.w, acc[(2 * h4 + 1) & 3]);
+          }
+        }
+        const float sum = (lo32(acc[0]) + hi32(acc[0])) + (lo32(acc[1]) + hi32(acc[1])) +
+                          ((lo32(acc[2]) + hi32(acc[2])) + (lo32(acc[3]) + hi32(acc[3])));
+        if (s < R.max_len) {
+          if (s <= ri.t)
+            o[s] = sum * ks;
+          else if (fill)
+            o[s] = -INFINITY;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_empty(slot));
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_empty(qb));
+      ++si;
+    } while (seg_next(R, row0, nrows, sg));
+    if (!ok) *abort_flag = 1;
   }
 
   tc_fence_before();
@@ -423,7 +739,7 @@ bool indexer_tc_supported(int dtype, int H_I, int D_I) {
   return (dtype == DSA_BF16 || dtype == DSA_E4M3) && H_I == kHI && D_I == kDI;
 }
 
-template <int DT, int G, int NG, int NK, bool DECODE>
+template <int DT, int G, int NG, int NK>
 static dsa_status_t launch_cfg(const Rows& R, int32_t row0, int32_t nrows, const void* q_idx,
                                const float* q_scale, const float* w, const void* k_idx,
                                const float* k_scale, float* scores, int64_t ld, bool fill,
@@ -436,19 +752,37 @@ static dsa_status_t launch_cfg(const Rows& R, int32_t row0, int32_t nrows, const
   if (!make_tmap_2d(&qmap, q_idx, tdt, C::ESZ, kDI, (uint64_t)R.n_q * kHI, box_cols, C::N) ||
       !make_tmap_2d(&kmap, k_idx, tdt, C::ESZ, kDI, (uint64_t)R.n_k, box_cols, kTileK))
     return DSA_ERR_CUDA;
-  auto kfn = indexer_tc_kernel<DT, G, NG, NK, DECODE>;
+  auto kfn = indexer_tc_kernel<DT, G, NG, NK>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
-  dim3 grid;
-  if (DECODE) {
-    grid = dim3((R.max_len + kDecodeChunk - 1) / kDecodeChunk, nrows);
-  } else {
-    const int32_t span = nrows < R.max_len ? nrows : R.max_len;
-    grid = dim3((span + C::QB - 1) / C::QB + 1, R.B);
-  }
+  const int32_t span = nrows < R.max_len ? nrows : R.max_len;
+  const dim3 grid((span + C::QB - 1) / C::QB + 1, R.B);
   kfn<<<grid, kThreads, C::SMEM, st>>>(qmap, kmap, R, row0, nrows, w, q_scale, k_scale, scores,
                                        ld, fill ? 1 : 0);
+  return launch_status();
+}
+
+template <int DT, int NK>
+static dsa_status_t launch_decode(const Rows& R, int32_t row0, int32_t nrows, const void* q_idx,
+                                  const float* q_scale, const float* w, const void* k_idx,
+                                  const float* k_scale, float* scores, int64_t ld, bool fill,
+                                  cudaStream_t st) {
+  using D = DecCfg<DT, NK>;
+  using C = typename D::C;
+  CUtensorMap qmap, kmap;
+  const CUtensorMapDataType tdt =
+      DT == DSA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const uint32_t box_cols = 128 / C::ESZ;
+  if (!make_tmap_2d(&qmap, q_idx, tdt, C::ESZ, kDI, (uint64_t)R.n_q * kHI, box_cols, C::N) ||
+      !make_tmap_2d(&kmap, k_idx, tdt, C::ESZ, kDI, (uint64_t)R.n_k, box_cols, kTileK))
+    return DSA_ERR_CUDA;
+  auto kfn = indexer_decode_kernel<DT, NK>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  kfn<<<num_sms(), kThreads, D::SMEM, st>>>(qmap, kmap, R, row0, nrows, w, q_scale, k_scale,
+                                            scores, ld, fill ? 1 : 0);
   return launch_status();
 }
 
@@ -461,15 +795,15 @@ dsa_status_t launch_indexer_tc(const Rows& R, int32_t row0, int32_t nrows, int d
   const bool decode = R.mode == DSA_DECODE;
   if (dtype == DSA_BF16) {
     if (decode)
-      return launch_cfg<DSA_BF16, 1, 1, 6, true>(R, row0, nrows, q_idx, q_scale, w, k_idx,
-                                                 k_scale, scores, ld, fill, st);
-    return launch_cfg<DSA_BF16, 4, 2, 2, false>(R, row0, nrows, q_idx, q_scale, w, k_idx,
+      return launch_decode<DSA_BF16, 6>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale, scores,
+                                        ld, fill, st);
+    return launch_cfg<DSA_BF16, 4, 2, 2>(R, row0, nrows, q_idx, q_scale, w, k_idx,
                                                 k_scale, scores, ld, fill, st);
   }
   if (decode)
-    return launch_cfg<DSA_E4M3, 1, 1, 8, true>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale,
-                                               scores, ld, fill, st);
-  return launch_cfg<DSA_E4M3, 4, 2, 4, false>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale,
+    return launch_decode<DSA_E4M3, 12>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale, scores,
+                                       ld, fill, st);
+  return launch_cfg<DSA_E4M3, 4, 2, 4>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale,
                                               scores, ld, fill, st);
 }
 

@@ -20,9 +20,11 @@
 //           written out at once (in any order), the members of b1 --
 //           typically a hundred or so -- go to a candidate buffer in shared
 //           memory with their fp32 keys.
-// The candidates are then ranked directly (key, then position: ties go to
-// the lower position) and the best k - |above b1| of them written out.  A
-// bin b1 with more members than the buffer holds is resolved by radix
+// The candidates are then split once more: a histogram of their keys over
+// 2048 buckets spanning the candidates' key range finds the bucket at the
+// cut, the buckets above it go out, and only that bucket's members (one or
+// two, typically) are ranked (key, then position: ties go to the lower
+// position) for the last of the k - |above b1| slots.  A bin b1 with more members than the buffer holds is resolved by radix
 // passes over the row instead (11 + 11 + 10 bits of the fp32 key), with
 // ties at the cut filled from the lowest positions by an ordered pass over
 // the row (ballot + warp prefix + a scan of warp totals).
@@ -36,6 +38,8 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kCand = 2048;  // candidate buffer (keys + positions)
+constexpr int kBatch = 4;    // float4 loads each thread keeps in flight per step
+constexpr int kBatchRow = 2;  // the same at three CTAs per SM (42 registers)
 
 __device__ __forceinline__ uint32_t rank_key(float x) {
   uint32_t u = __float_as_uint(x);
@@ -77,6 +81,7 @@ struct Smem {
   uint32_t sel_above;
   uint32_t n_out;   // positions written so far
   uint32_t n_cand;  // members of bin b1 seen in pass 2
+  uint32_t kmin, kmax;  // candidate key range (ranking)
 };
 
 // Given hist[0..nbins) and the number `need` of elements still to take,
@@ -122,21 +127,91 @@ __device__ __forceinline__ uint32_t warp_append(bool pred, uint32_t* ctr, uint32
   return mask;
 }
 
-// Writes the `need` best of m candidates (key, position) to dst[0 .. need):
-// rank = candidates with a larger key, or an equal key at a lower position
-// (the tie rule), and candidate j goes to dst[rank] when rank < need.  All
-// threads of the CTA call it.
-__device__ void rank_candidates(const uint32_t* ckey, const int32_t* cpos, int m, uint32_t need,
+// Order of candidates: a larger key first, then (the tie rule) the lower
+// position.  Positions are distinct, so no two candidates compare equal.
+__device__ __forceinline__ uint64_t cand_order(uint32_t key, int32_t pos) {
+  return ((uint64_t)key << 32) | (uint64_t)(0xffffffffu - (uint32_t)pos);
+}
+
+__device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Writes the `need` best of m <= kCand candidates (key, position) to
+// dst[0 .. need) in any order.  The candidates' keys span [kmin, kmax]; a
+// histogram of (key - kmin) >> shift over kBins buckets (monotone in the key)
+// finds the bucket sb that holds the need-th best.  Candidates in buckets
+// above sb go out at once; the members of sb (typically one or two) move to
+// the front of the candidate arrays and are ranked by the candidate order,
+// one warp per member with its lanes sharing the comparisons, the best of
+// them filling the remaining slots.  All threads of the CTA call it.
+__device__ void rank_candidates(Smem& sm, uint32_t* ckey, int32_t* cpos, int m, uint32_t need,
                                 int32_t* dst) {
-  for (int j = threadIdx.x; j < m; j += kThreads) {
-    const uint32_t kj = ckey[j];
-    const int32_t pj = cpos[j];
-    uint32_t rank = 0;
-    for (int l = 0; l < m; ++l) {
-      const uint32_t kl = ckey[l];
-      rank += (kl > kj || (kl == kj && cpos[l] < pj)) ? 1u : 0u;
+  constexpr int R = kCand / kThreads;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t key[R];
+  int32_t pos[R];
+  uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int j = tid + r * kThreads;
+    key[r] = j < m ? ckey[j] : 0u;
+    pos[r] = j < m ? cpos[j] : 0;
+    if (j < m) {
+      lo = min(lo, key[r]);
+      hi = max(hi, key[r]);
     }
-    if (rank < need) dst[rank] = pj;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (tid == 0) {
+    sm.kmin = 0xffffffffu;
+    sm.kmax = 0u;
+    sm.n_out = 0;
+    sm.n_cand = 0;
+  }
+  for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0;
+  __syncthreads();
+  if (lane == 0) {
+    atomicMin(&sm.kmin, lo);
+    atomicMax(&sm.kmax, hi);
+  }
+  __syncthreads();
+  const uint32_t kmin = sm.kmin, span = sm.kmax - kmin;
+  const int bits = span ? 32 - __clz(span) : 0;  // bits of the span
+  const int shift = bits > 11 ? bits - 11 : 0;   // (span >> shift) < 2048 buckets
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    if (tid + r * kThreads < m) atomicAdd(&sm.hist[(key[r] - kmin) >> shift], 1u);
+  __syncthreads();
+  find_bin(sm, kBins, need);  // ends with a barrier: every candidate is in registers
+  const uint32_t sb = sm.sel_bin, need2 = need - sm.sel_above;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const bool ok = tid + r * kThreads < m;
+    const uint32_t b = (key[r] - kmin) >> shift;
+    const bool up = ok && b > sb, in = ok && b == sb;
+    uint32_t slot;
+    if (warp_append(up, &sm.n_out, slot) && up) dst[slot] = pos[r];
+    if (warp_append(in, &sm.n_cand, slot) && in) {
+      ckey[slot] = key[r];
+      cpos[slot] = pos[r];
+    }
+  }
+  __syncthreads();
+  const int c = (int)sm.n_cand;
+  const uint32_t base_out = sm.n_out;  // == sm.sel_above
+  for (int j = warp; j < c; j += kWarps) {
+    const uint64_t oj = cand_order(ckey[j], cpos[j]);
+    uint32_t better = 0;
+    for (int l = lane; l < c; l += 32) better += cand_order(ckey[l], cpos[l]) > oj ? 1u : 0u;
+    better = warp_sum(better);
+    if (lane == 0 && better < need2) dst[base_out + better] = cpos[j];
   }
 }
 
@@ -213,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(Rows R, int32_t row0,
   __shared__ uint32_t ckey[kCand];
   __shared__ int32_t cpos[kCand];
   __shared__ Smem sm;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int32_t r = row0 + blockIdx.x;
   const RowInfo ri = row_info(R, r);
   const int n = ri.t + 1;
@@ -223,8 +298,14 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(Rows R, int32_t row0,
     return;
   }
   const float* row = scores + (int64_t)blockIdx.x * ld;
-  // Rows start 16-byte aligned when ld is a multiple of 4 (the buffer itself is).
-  const bool vec = (ld & 3) == 0;
+  // The row as a scalar head up to the first 16-byte boundary, n4 float4
+  // vectors from a0, and a scalar tail from t0 (row strides need not be
+  // multiples of four floats).
+  const int a0 =
+      min(n, (int)((4u - (uint32_t)((reinterpret_cast<uintptr_t>(row) >> 2) & 3u)) & 3u));
+  const int n4 = (n - a0) >> 2, t0 = a0 + 4 * n4;
+  const int n_head = a0, n_edge = n_head + (n - t0);  // <= 6 scalar scores
+  const float4* row4 = reinterpret_cast<const float4*>(row + a0);
 
   // ------------------------------------------------------------ pass 1
   for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0;
@@ -233,19 +314,25 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(Rows R, int32_t row0,
     sm.n_cand = 0;
   }
   __syncthreads();
-  const float4* row4 = reinterpret_cast<const float4*>(row);
-  const int n4 = (n + 3) >> 2;  // the last vector may run past n (not past ld)
-  if (vec) {
-#pragma unroll 4
-    for (int v = tid; v < n4; v += kThreads) {
-      const float4 x = __ldg(row4 + v);
-      const float xs[4] = {x.x, x.y, x.z, x.w};
+  if (tid < n_edge) {
+    const int i = tid < n_head ? tid : t0 + (tid - n_head);
+    atomicAdd(&sm.hist[score_bin(__ldg(row + i))], 1u);
+  }
+  for (int base = tid; base < n4; base += kBatchRow * kThreads) {
+    float4 xv[kBatchRow];
+#pragma unroll
+    for (int u = 0; u < kBatchRow; ++u) {
+      const int v = base + u * kThreads;
+      if (v < n4) xv[u] = __ldg(row4 + v);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatchRow; ++u) {
+      const int v = base + u * kThreads;
+      const float xs[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        if (4 * v + e < n) atomicAdd(&sm.hist[score_bin(xs[e])], 1u);
+        if (v < n4) atomicAdd(&sm.hist[score_bin(xs[e])], 1u);
     }
-  } else {
-    for (int i = tid; i < n; i += kThreads) atomicAdd(&sm.hist[score_bin(__ldg(row + i))], 1u);
   }
   __syncthreads();
   find_bin(sm, kBins, (uint32_t)k);
@@ -257,26 +344,55 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(Rows R, int32_t row0,
 
   // ------------------------------------------------------------ pass 2
   // Everything above b1 is selected; the members of b1 become candidates
-  // (when they all fit the buffer).
+  // (when they all fit the buffer).  b1 is the float interval [lo, hi]; the
+  // -inf bin 0 holds NaN too, which no float comparison admits, so bins are
+  // compared there.
   const bool collect = in_b1 <= (uint32_t)kCand;
   float lo, hi;
   bin_bounds(b1, lo, hi);
-  if (vec && b1 != 0) {
-    // four scores per thread: above hi -> written out (one atomic per warp
-    // and step), in [lo, hi] -> candidates (rare: per-score appends)
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int base = 0; base < n4; base += kThreads) {  // uniform trip count
-      const int v = base + tid;
-      const float4 x = v < n4 ? __ldg(row4 + v) : make_float4(-INFINITY, -INFINITY, -INFINITY,
-                                                              -INFINITY);
-      const float xs[4] = {x.x, x.y, x.z, x.w};
+  auto classify = [&](float x, bool valid, bool& gt, bool& eq) {
+    if (b1 != 0) {
+      gt = valid && x > hi;
+      eq = valid && !gt && x >= lo;
+    } else {
+      const uint32_t b = valid ? score_bin(x) : 0u;
+      gt = valid && b > b1;
+      eq = valid && b == b1;
+    }
+    eq = eq && collect;
+  };
+  if (tid < 32) {  // the scalar head and tail in warp 0
+    const bool mine = tid < n_edge;
+    const int i = tid < n_head ? tid : t0 + (tid - n_head);
+    const float x = mine ? __ldg(row + i) : 0.f;
+    bool gt, eq;
+    classify(x, mine, gt, eq);
+    uint32_t slot;
+    if (warp_append(gt, &sm.n_out, slot) && gt) out[slot] = i;
+    if (warp_append(eq, &sm.n_cand, slot) && eq) {
+      ckey[slot] = rank_key(x);
+      cpos[slot] = i;
+    }
+  }
+  // four scores per vector: above b1 -> written out (one atomic per warp and
+  // vector), members of b1 -> candidates (rare: per-score appends)
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int base = 0; base < n4; base += kBatchRow * kThreads) {  // uniform trip count
+    float4 xv[kBatchRow];
+#pragma unroll
+    for (int u = 0; u < kBatchRow; ++u) {
+      const int v = base + u * kThreads + tid;
+      xv[u] = v < n4 ? __ldg(row4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatchRow; ++u) {
+      const int v = base + u * kThreads + tid;
+      const float xs[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
       bool gt[4], eq[4];
       bool any_eq = false;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const bool ok = 4 * v + e < n;
-        gt[e] = ok && xs[e] > hi;
-        eq[e] = ok && !gt[e] && xs[e] >= lo;
+        classify(xs[e], v < n4, gt[e], eq[e]);
         any_eq |= eq[e];
       }
       uint32_t g[4], tot = 0;
@@ -291,39 +407,26 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(Rows R, int32_t row0,
         slot = __shfl_sync(0xffffffffu, slot, 0);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          if (gt[e]) out[slot + __popc(g[e] & lt)] = 4 * v + e;
+          if (gt[e]) out[slot + __popc(g[e] & lt)] = a0 + 4 * v + e;
           slot += __popc(g[e]);
         }
       }
-      if (collect && __any_sync(0xffffffffu, any_eq)) {
+      if (__any_sync(0xffffffffu, any_eq)) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           uint32_t slot;
           if (warp_append(eq[e], &sm.n_cand, slot) && eq[e]) {
             ckey[slot] = rank_key(xs[e]);
-            cpos[slot] = 4 * v + e;
+            cpos[slot] = a0 + 4 * v + e;
           }
         }
-      }
-    }
-  } else {
-    for (int base = 0; base < n; base += kThreads) {  // uniform trip count
-      const int i = base + tid;
-      const float x = i < n ? __ldg(row + i) : 0.f;
-      const uint32_t b = i < n ? score_bin(x) : 0u;
-      const bool gt = i < n && b > b1, eq = collect && i < n && b == b1;
-      uint32_t slot;
-      if (warp_append(gt, &sm.n_out, slot) && gt) out[slot] = i;
-      if (warp_append(eq, &sm.n_cand, slot) && eq) {
-        ckey[slot] = rank_key(x);
-        cpos[slot] = i;
       }
     }
   }
   __syncthreads();
 
   if (collect) {
-    rank_candidates(ckey, cpos, (int)in_b1, need, out + above1);
+    rank_candidates(sm, ckey, cpos, (int)in_b1, need, out + above1);
     return;
   }
 
@@ -332,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(Rows R, int32_t row0,
 
 // ---------------------------------------------------------------- split rows
 // Few long rows (decode) leave most SMs idle with one CTA per row, so each
-// row is split over a cluster of kParts CTAs.  Each histograms its slice;
+// row is split over a cluster of P CTAs.  Each histograms its slice;
 // the slices' histograms are summed into the leader's (CTA 0) through
 // distributed shared memory (a reduction per non-empty bin), and the leader
 // fixes b1.  Each CTA then filters its slice into local buffers -- scores
@@ -340,7 +443,6 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(Rows R, int32_t row0,
 // leader's counters, writes its scores above b1 to the output and its
 // candidates into the leader's buffer.  The leader ranks the candidates (or
 // resolves an overflowing b1 from the row) exactly as the one-CTA kernel.
-constexpr int kParts = 4;
 
 __device__ __forceinline__ uint32_t cl_rank() {
   uint32_t r;
@@ -375,7 +477,8 @@ __device__ __forceinline__ void cl_st(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-__global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads, 2)
+template <int P>
+__global__ void __cluster_dims__(P, 1, 1) __launch_bounds__(kThreads, 2)
     topk_split_kernel(Rows R, int32_t row0, const float* scores, int64_t ld, int k,
                       int32_t* idx) {
   extern __shared__ uint32_t dyn[];
@@ -387,9 +490,9 @@ __global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads, 2)
   __shared__ Smem sm;
   __shared__ uint32_t info[4];  // leader: b1, above1, |b1|; every CTA: its two reservations
   __shared__ uint32_t local_gt, local_cand;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t crank = cl_rank();
-  const int32_t rloc = blockIdx.x / kParts;
+  const int32_t rloc = blockIdx.x / P;
   const RowInfo ri = row_info(R, row0 + rloc);
   const int n = ri.t + 1;
   int32_t* out = idx + (int64_t)rloc * k;
@@ -399,9 +502,16 @@ __global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads, 2)
     return;
   }
   const float* row = scores + (int64_t)rloc * ld;
-  const bool vec = (ld & 3) == 0;
-  const int chunk = ((n + kParts - 1) / kParts + 3) & ~3;  // slices start 16-byte aligned
+  const int chunk = ((n + P - 1) / P + 3) & ~3;
   const int p0 = min(n, (int)crank * chunk), p1 = min(n, p0 + chunk);
+  // The slice as a scalar head up to the first 16-byte boundary, m4 float4
+  // vectors from a0, and a scalar tail from t0 (row strides need not be
+  // multiples of four floats).
+  const int a0 = min(
+      p1, p0 + (int)((4u - (uint32_t)((reinterpret_cast<uintptr_t>(row + p0) >> 2) & 3u)) & 3u));
+  const int m4 = (p1 - a0) >> 2, t0 = a0 + 4 * m4;
+  const int n_head = a0 - p0, n_edge = n_head + (p1 - t0);  // <= 6 scalar scores
+  const float4* s4 = reinterpret_cast<const float4*>(row + a0);
 
   // ------------------------------------------------------------ slice histogram
   for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0;
@@ -412,19 +522,25 @@ __global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads, 2)
     local_cand = 0;
   }
   __syncthreads();
-  if (vec) {
-    const float4* s4 = reinterpret_cast<const float4*>(row + p0);
-    const int m4 = (p1 - p0 + 3) >> 2;
-#pragma unroll 4
-    for (int v = tid; v < m4; v += kThreads) {
-      const float4 x = __ldg(s4 + v);
-      const float xs[4] = {x.x, x.y, x.z, x.w};
+  if (tid < n_edge) {
+    const int i = tid < n_head ? p0 + tid : t0 + (tid - n_head);
+    atomicAdd(&sm.hist[score_bin(__ldg(row + i))], 1u);
+  }
+  for (int base = tid; base < m4; base += kBatch * kThreads) {
+    float4 xv[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int v = base + u * kThreads;
+      if (v < m4) xv[u] = __ldg(s4 + v);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int v = base + u * kThreads;
+      const float xs[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        if (p0 + 4 * v + e < p1) atomicAdd(&sm.hist[score_bin(xs[e])], 1u);
+        if (v < m4) atomicAdd(&sm.hist[score_bin(xs[e])], 1u);
     }
-  } else {
-    for (int i = p0 + tid; i < p1; i += kThreads) atomicAdd(&sm.hist[score_bin(__ldg(row + i))], 1u);
   }
   __syncthreads();
   cl_sync();  // every slice histogram complete
@@ -465,37 +581,72 @@ __global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads, 2)
     }
     eq = eq && collect;
   };
-  if (vec) {
-    const float4* s4 = reinterpret_cast<const float4*>(row + p0);
-    const int m4 = (p1 - p0 + 3) >> 2;
-    for (int base = 0; base < m4; base += kThreads) {  // uniform trip count
-      const int v = base + tid;
-      const float4 x = v < m4 ? __ldg(s4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float xs[4] = {x.x, x.y, x.z, x.w};
+  // the scalar head and tail (at most six scores) in warp 0
+  if (tid < 32) {
+    const bool mine = tid < n_edge;
+    const int i = tid < n_head ? p0 + tid : t0 + (tid - n_head);
+    const float x = mine ? __ldg(row + i) : 0.f;
+    bool gt, eq;
+    classify(x, mine, gt, eq);
+    uint32_t slot;
+    if (warp_append(gt, &local_gt, slot) && gt) gpos[slot] = i;
+    if (warp_append(eq, &local_cand, slot) && eq) {
+      ckey[slot] = rank_key(x);
+      cpos[slot] = i;
+    }
+  }
+  for (int base = 0; base < m4; base += kBatch * kThreads) {  // uniform trip count
+    float4 xv[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int v = base + u * kThreads + tid;
+      xv[u] = v < m4 ? __ldg(s4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // classify the batch into two bit masks, then reserve the slots of the
+    // whole warp's batch with one atomic per list (lane 0), the lanes
+    // taking consecutive ranges by a prefix sum of their counts
+    uint32_t gtm = 0, eqm = 0;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int v = base + u * kThreads + tid;
+      const float xs[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int i = p0 + 4 * v + e;
         bool gt, eq;
-        classify(xs[e], v < m4 && i < p1, gt, eq);
-        uint32_t slot;
-        if (warp_append(gt, &local_gt, slot) && gt) gpos[slot] = i;  // < above1 < k <= kCand
-        if (warp_append(eq, &local_cand, slot) && eq) {
-          ckey[slot] = rank_key(xs[e]);
-          cpos[slot] = i;
-        }
+        classify(xs[e], v < m4, gt, eq);
+        gtm |= (gt ? 1u : 0u) << (4 * u + e);
+        eqm |= (eq ? 1u : 0u) << (4 * u + e);
       }
     }
-  } else {
-    for (int base = p0; base < p1; base += kThreads) {  // uniform trip count
-      const int i = base + tid;
-      const float x = i < p1 ? __ldg(row + i) : 0.f;
-      bool gt, eq;
-      classify(x, i < p1, gt, eq);
-      uint32_t slot;
-      if (warp_append(gt, &local_gt, slot) && gt) gpos[slot] = i;
-      if (warp_append(eq, &local_cand, slot) && eq) {
-        ckey[slot] = rank_key(x);
-        cpos[slot] = i;
+    const uint32_t own = (uint32_t)__popc(gtm) | ((uint32_t)__popc(eqm) << 16);
+    uint32_t incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+    if (!tot) continue;  // warp-uniform
+    uint32_t wb = 0;
+    if (lane == 0) {
+      const uint32_t bg = (tot & 0xffffu) ? atomicAdd(&local_gt, tot & 0xffffu) : 0u;
+      const uint32_t be = (tot >> 16) ? atomicAdd(&local_cand, tot >> 16) : 0u;
+      wb = bg | (be << 16);  // both below kCand
+    }
+    wb = __shfl_sync(0xffffffffu, wb, 0) + (incl - own);
+    uint32_t sg = wb & 0xffffu, se = wb >> 16;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int v = base + u * kThreads + tid;
+      const float xs[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = a0 + 4 * v + e;
+        if ((gtm >> (4 * u + e)) & 1u) gpos[sg++] = i;  // < above1 < k <= kCand
+        if ((eqm >> (4 * u + e)) & 1u) {
+          ckey[se] = rank_key(xs[e]);
+          cpos[se++] = i;
+        }
       }
     }
   }
@@ -516,7 +667,7 @@ __global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads, 2)
 
   if (crank == 0) {
     if (collect)
-      rank_candidates(mkey, mpos, (int)in_b1, (uint32_t)k - above1, out + above1);
+      rank_candidates(sm, mkey, mpos, (int)in_b1, (uint32_t)k - above1, out + above1);
     else
       resolve_by_row(sm, row, n, k, b1, above1, out);  // sm.n_out == above1 here
   }
@@ -527,14 +678,17 @@ __global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads, 2)
 dsa_status_t launch_topk(const Rows& R, int32_t row0, int32_t nrows, const float* scores,
                          int64_t ld, int k, int32_t* idx, cudaStream_t st) {
   if (nrows <= 0) return DSA_OK;
-  // Few long rows: one cluster of kParts CTAs per row; otherwise one CTA per
-  // row, several per SM.
-  if (k <= kCand && nrows * kParts <= 4 * num_sms() && R.max_len >= 8 * k) {
+  // Few long rows: one cluster of 4 or 8 CTAs per row (8 while all the
+  // clusters fit one wave at two CTAs per SM); otherwise one CTA per row,
+  // several per SM.
+  if (k <= kCand && nrows * 4 <= 4 * num_sms() && R.max_len >= 8 * k) {
     const size_t smem = 4 * kCand * sizeof(uint32_t);  // + static: above the 48 KB default
-    if (cudaFuncSetAttribute(topk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    const bool eight = nrows * 8 <= 2 * num_sms() && R.max_len >= 16 * k;
+    auto kfn = eight ? topk_split_kernel<8> : topk_split_kernel<4>;
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
       return DSA_ERR_CUDA;
-    topk_split_kernel<<<nrows * kParts, kThreads, smem, st>>>(R, row0, scores, ld, k, idx);
+    kfn<<<nrows * (eight ? 8 : 4), kThreads, smem, st>>>(R, row0, scores, ld, k, idx);
     return launch_status();
   }
   topk_kernel<<<nrows, kThreads, 0, st>>>(R, row0, scores, ld, k, idx);

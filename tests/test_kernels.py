@@ -17,12 +17,19 @@ from dsa_testutil import (Dev, assert_attn_close, assert_scores_close, ref_attn,
 
 pytestmark = pytest.mark.gpu
 
+# 48 decode rows: lengths 1..3000 with a run of rows of at most one key tile
+_MANY = [(i * 2654435761) % 2999 + 1 for i in range(32)] + [1, 7, 128, 129, 64, 2, 100, 3] * 2
+
 SMALL = {
     "c1_tiny_f32": workloads.config(1),
     "prefill_bf16_ragged": workloads.custom("prefill", [300, 45, 129], idx_dtype="bf16", k=64),
     "prefill_e4m3": workloads.custom("prefill", [333], idx_dtype="e4m3", k=100),
     "decode_bf16": workloads.custom("decode", [1, 200, 700, 129], idx_dtype="bf16", k=128),
     "decode_e4m3": workloads.custom("decode", [2049, 5, 4100], idx_dtype="e4m3", k=2048),
+    # enough key tiles that the persistent decode indexer gives each CTA a
+    # range crossing several rows, runs of one-tile rows among them
+    "decode_bf16_many_rows": workloads.custom("decode", _MANY, idx_dtype="bf16", k=64),
+    "decode_e4m3_many_rows": workloads.custom("decode", _MANY[::-1], idx_dtype="e4m3", k=96),
     "prefill_f32_generic_dims": workloads.custom("prefill", [150], H_I=16, D_I=64,
                                                  idx_dtype="f32", k=20, H=20, D_K=96, D_V=32),
 }
@@ -76,11 +83,16 @@ def _decode_layout(lens):
     return dsa.Layout(d, dsa.DSA_DECODE, max(lens), len(lens), int(offs[-1]))
 
 
-def test_topk_edge_rows():
+@pytest.mark.parametrize("odd_stride", [False, True])
+def test_topk_edge_rows(odd_stride):
     """Rows shorter than, equal to and one longer than k; all-equal rows;
-    -0/+0 ties; NaN; rows longer than the shared-memory cache (131072)."""
+    -0/+0 ties; NaN; rows of 131072.  With odd_stride a last row of 131075
+    makes the row stride 131075 floats, so no row after the first starts on
+    a 16-byte boundary."""
     k = 2048
     lens = [1, 100, k, k + 1, 5000, 5000, 5000, 60000, 131072, 131072]
+    if odd_stride:
+        lens.append(131075)
     L = _decode_layout(lens)
     g = torch.Generator().manual_seed(5)
     S = torch.randn(len(lens), max(lens), generator=g)
@@ -89,7 +101,7 @@ def test_topk_edge_rows():
     S[5, :] = 0.0
     S[5, ::2] = -0.0  # +0 and -0 everywhere: lowest positions win
     S[6, 100:200] = float("nan")
-    S[9] = torch.arange(131072, dtype=torch.float32).flip(0) * 1e-3  # strictly decreasing
+    S[9, :131072] = torch.arange(131072, dtype=torch.float32).flip(0) * 1e-3  # decreasing
     dS = S.cuda()
     idx = torch.empty(len(lens), k, dtype=torch.int32, device="cuda")
     dsa.dsa_topk(L, dS, k, idx)
