@@ -10,7 +10,10 @@ decode batch (64 sequences, lengths 4K..64K, bf16 indexer), measured the same
 way.
 
 Timing: W untimed warm-up steps, then K steps, each preceded by an L2 flush
-(a 512 MB write) outside its CUDA-event interval; barrier + synchronize
+outside its CUDA-event interval: a 512 MB write, then a read of 256 MB of
+it, so that the step starts with none of the previous step's lines in L2
+and no dirty line either (write-backs of the flush would otherwise take
+about 20 us of HBM time from the first kernel of the step); barrier + synchronize
 around the timed region; the max over ranks.  Multi-GPU runs are weak
 scaling: every rank processes its own copy of the workload (independent
 sequences), no collective on the data path.
@@ -199,6 +202,7 @@ def run_device(cid, steps, warmup, rank, world, do_e2e=True):
     time.sleep(0.3)
     for i in range(steps):
         flush.fill_(float(i))
+        flush[: 64 << 20].sum()  # 256 MB read: the write-backs happen here
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         kinds, nl = step(evs)
@@ -474,7 +478,7 @@ def main():
             "dtype": {"f32": "f32", "bf16": "bf16", "e4m3": "e4m3+bf16"}[cfg.idx_dtype],
             "data": "synthetic",
             "config": {"workload": DESCR[cid], "tokens_per_step_per_gpu": tokens,
-                       "k": cfg.k, "l2": "flushed before every timed step (512 MB write)",
+                       "k": cfg.k, "l2": "flushed before every timed step (512 MB write, 256 MB of it read back)",
                        "parallelism": f"{world} independent replicas (weak scaling)"},
             "roofline": roof, "stage_share": shares,
             "gpu_launches": launches,
