@@ -59,6 +59,47 @@ __device__ __forceinline__ uint64_t fma2(float x0, float x1, float w0, float w1,
 __device__ __forceinline__ float lo32(uint64_t v) { return __uint_as_float((uint32_t)v); }
 __device__ __forceinline__ float hi32(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
 
+// Weighted ReLU head sum of one key for one query: the 64 fp32 head scores
+// at TMEM columns ta .. ta+63 of this warp's lanes, weights w[0..63] in
+// shared memory.  Both 32-column loads are in flight before the one wait.
+__device__ __forceinline__ float relu_wsum(uint32_t ta, const float4* __restrict__ wr) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+        "=r"(r[62]), "=r"(r[63])
+      : "r"(ta), "r"(ta + 32)
+      : "memory");
+  uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int h4 = 0; h4 < 16; ++h4) {
+    const float4 w4 = wr[h4];
+    acc[(2 * h4) & 3] = fma2(fmaxf(__uint_as_float(r[4 * h4]), 0.f),
+                             fmaxf(__uint_as_float(r[4 * h4 + 1]), 0.f), w4.x, w4.y,
+                             acc[(2 * h4) & 3]);
+    acc[(2 * h4 + 1) & 3] = fma2(fmaxf(__uint_as_float(r[4 * h4 + 2]), 0.f),
+                                 fmaxf(__uint_as_float(r[4 * h4 + 3]), 0.f), w4.z, w4.w,
+                                 acc[(2 * h4 + 1) & 3]);
+  }
+  return (lo32(acc[0]) + hi32(acc[0])) + (lo32(acc[1]) + hi32(acc[1])) +
+         ((lo32(acc[2]) + hi32(acc[2])) + (lo32(acc[3]) + hi32(acc[3])));
+}
+
 template <int DT, int G, int NG, int NK>
 struct Cfg {
   static constexpr int ESZ = DT == DSA_BF16 ? 2 : 1;
@@ -294,22 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int qi = g * G + qq;
             const float4* wr = reinterpret_cast<const float4*>(wq + qi * kHI);
             const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + slot * C::N + qq * kHI;
-            uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              float v[32];
-              tmem_ld32(ta + 32 * half, v);
-#pragma unroll
-              for (int h4 = 0; h4 < 8; ++h4) {
-                const float4 w4 = wr[8 * half + h4];
-                acc[(2 * h4) & 3] = fma2(fmaxf(v[4 * h4], 0.f), fmaxf(v[4 * h4 + 1], 0.f), w4.x,
-                                         w4.y, acc[(2 * h4) & 3]);
-                acc[(2 * h4 + 1) & 3] = fma2(fmaxf(v[4 * h4 + 2], 0.f), fmaxf(v[4 * h4 + 3], 0.f),
-                                             w4.z, w4.w, acc[(2 * h4 + 1) & 3]);
-              }
-            }
-            const float sum = (lo32(acc[0]) + hi32(acc[0])) + (lo32(acc[1]) + hi32(acc[1])) +
-                              ((lo32(acc[2]) + hi32(acc[2])) + (lo32(acc[3]) + hi32(acc[3])));
+            const float sum = relu_wsum(ta, wr);
             const int32_t tq = wk.t0 + qi;
             if (tq >= wk.qvalid_lo && tq < wk.qvalid_hi && s < R.max_len) {
               float* o = scores + (int64_t)(wk.qrow0 + qi - row0) * ld;
@@ -669,22 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + slot * C::N;
-        uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float v[32];
-          tmem_ld32(ta + 32 * half, v);
-#pragma unroll
-          for (int h4 = 0; h4 < 8; ++h4) {
-            const float4 w4 = wr[8 * half + h4];
-            acc[(2 * h4) & 3] = fma2(fmaxf(v[4 * h4], 0.f), fmaxf(v[4 * h4 + 1], 0.f), w4.x, w4.y,
-                                     acc[(2 * h4) & 3]);
-            acc[(2 * h4 + 1) & 3] = fma2(fmaxf(v[4 * h4 + 2], 0.f), fmaxf(v[4 * h4 + 3], 0.f),
-                                         w4.z, w4.w, acc[(2 * h4 + 1) & 3]);
-          }
-        }
-        const float sum = (lo32(acc[0]) + hi32(acc[0])) + (lo32(acc[1]) + hi32(acc[1])) +
-                          ((lo32(acc[2]) + hi32(acc[2])) + (lo32(acc[3]) + hi32(acc[3])));
+        const float sum = relu_wsum(ta, wr);
         if (s < R.max_len) {
           if (s <= ri.t)
             o[s] = sum * ks;
