@@ -224,6 +224,20 @@ dsa_status_t dsa_forward_timed(const dsa_layout_t* layout, const dsa_forward_arg
  */
 dsa_status_t dsa_device_status(void* stream);
 
+/*
+ * Self-test of the failure path every kernel shares: one thread waits on a
+ * barrier that nothing completes, using the same bounded wait as the
+ * kernels, but giving up after `cycles` clock cycles (0 .. the kernels' own
+ * limit of 2e9) instead of the kernels' limit.  The wait then raises the
+ * timeout bit, so the next dsa_device_status() returns DSA_ERR_TIMEOUT and
+ * the device stays usable.  No copy, MMA or other work is in flight when the
+ * wait gives up.  Not part of the method; it exists so that tests can see a
+ * wait run out without faulting or hanging the GPU.
+ * Returns DSA_ERR_INVALID_ARGUMENT for `cycles` outside that range,
+ * DSA_ERR_CUDA if the launch fails.
+ */
+dsa_status_t dsa_selftest_wait_timeout(int64_t cycles, void* stream);
+
 /* Static description of a status code. */
 const char* dsa_status_string(dsa_status_t status);
 

@@ -77,12 +77,13 @@ def lib():
         L.dsa_forward.argtypes = [LP, AP, P, P, P, P, SZ, P]
         L.dsa_forward_timed.argtypes = [LP, AP, P, P, P, P, SZ, P, P, I32, P, P]
         L.dsa_device_status.argtypes = [P]
+        L.dsa_selftest_wait_timeout.argtypes = [I64, P]
         L.dsa_status_string.argtypes = [ctypes.c_int]
         L.dsa_status_string.restype = ctypes.c_char_p
         L.dsa_abi_version.restype = I32
         for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn",
                      "dsa_sparse_mla_attn_noalloc", "dsa_forward",
-                     "dsa_forward_timed", "dsa_device_status"):
+                     "dsa_forward_timed", "dsa_device_status", "dsa_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -225,6 +226,12 @@ def dsa_forward_timed(layout: Layout, args: dsa_forward_args_t, out, lse, idx_ou
                                    _ptr(idx_out), _ptr(workspace), ws_bytes, _stream(stream), arr,
                                    n, kinds, ctypes.byref(nl)), "dsa_forward_timed")
     return [kinds[i] for i in range(min(nl.value, max(n - 1, 0)))], nl.value
+
+
+def dsa_selftest_wait_timeout(cycles: int, stream=None):
+    """Enqueues a wait on a barrier nothing completes, giving up after `cycles`."""
+    _check(lib().dsa_selftest_wait_timeout(int(cycles), _stream(stream)),
+           "dsa_selftest_wait_timeout")
 
 
 def dsa_device_status(stream=None) -> int:

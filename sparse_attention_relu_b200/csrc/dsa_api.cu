@@ -3,6 +3,7 @@
 #include <math.h>
 
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 namespace dsa {
 
@@ -24,6 +25,17 @@ unsigned* status_word() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// One thread waits, through the bounded wait every kernel uses, on an
+// mbarrier that nothing arrives on; after `limit` cycles the wait gives up
+// and raises kErrTimeout.  Nothing is in flight when it returns.
+__global__ void wait_timeout_selftest(unsigned* status, long long limit) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = (uint32_t)__cvta_generic_to_shared(&bar);
+  sm100::mbar_init(b, 1);
+  sm100::fence_mbar_init();
+  sm100::mbar_wait_for(b, 0, status, limit);
+}
 
 // Checks the layout; fills the device-side row description.
 dsa_status_t check_layout(const dsa_layout_t* L, Rows* R) {
@@ -186,6 +198,14 @@ dsa_status_t dsa_device_status(void* stream) {
   if (v & kErrTimeout) return DSA_ERR_TIMEOUT;
   if (v) return DSA_ERR_DEVICE_DATA;
   return DSA_OK;
+}
+
+dsa_status_t dsa_selftest_wait_timeout(int64_t cycles, void* stream) {
+  if (cycles < 0 || cycles > (int64_t)sm100::kSpinLimit) return DSA_ERR_INVALID_ARGUMENT;
+  unsigned* status = status_word();
+  if (!status) return DSA_ERR_CUDA;
+  wait_timeout_selftest<<<1, 1, 0, (cudaStream_t)stream>>>(status, (long long)cycles);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 dsa_status_t dsa_indexer_scores(const dsa_layout_t* layout, const void* q_idx,

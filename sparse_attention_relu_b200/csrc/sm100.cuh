@@ -64,17 +64,22 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kSpinLimit cycles, raising kErrTimeout in the status word; returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status) {
+// `limit` cycles, raising kErrTimeout in the status word; returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, unsigned* status,
+                                              long long limit) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try(bar, parity)) {
-    if (clock64() - t0 > kSpinLimit) {
+    if (clock64() - t0 > limit) {
       atomicOr(status, kErrTimeout);
       return false;
     }
   }
   return true;
+}
+// The wait every kernel uses: kSpinLimit cycles (about a second).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status) {
+  return mbar_wait_for(bar, parity, status, kSpinLimit);
 }
 
 // ---------------------------------------------------------------- TMA

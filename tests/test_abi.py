@@ -78,6 +78,9 @@ def test_argument_validation_without_device(lib):
     assert f(ctypes.byref(L), P, P, P, 4, 129, 576, 512, 0.1, P, None, None, 0, None) == E
     assert f(ctypes.byref(L), P, P, P, 4, 128, 576, 580, 0.1, P, None, None, 0, None) == E
     assert f(ctypes.byref(L), P, P, P, 4, 8, 80, 64, float("nan"), P, None, None, 0, None) == E
+    # the wait-timeout self-test takes limits in 0 .. 2e9 cycles only
+    assert lib.dsa_selftest_wait_timeout(-1, None) == E
+    assert lib.dsa_selftest_wait_timeout(2_000_000_001, None) == E
     # empty problems succeed without launching anything
     empty = _layout(batch=0, kv_offsets=None, max_len=0, n_q=0, n_k=0)
     assert lib.dsa_topk(ctypes.byref(empty), None, 4, None, None) == dsa.DSA_OK
