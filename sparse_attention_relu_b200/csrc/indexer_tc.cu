@@ -13,12 +13,12 @@
 // with no shuffles.  fp8 scales fold in for free: q_scale (positive) moves
 // into w, k_scale multiplies the finished sum.
 //
-// Warp roles (576 threads):
+// Warp roles (prefill: 832 threads):
 //   warp 0      TMA producer: the query block once, then a ring of key tiles
 //   warp 1      TMEM allocator and MMA issuer (one thread)
-//   warps 2-17  epilogue: TMEM -> registers, ReLU, weighted head sum, store.
-//               Four sets of four warps (one warp per TMEM lane quadrant in
-//               each) take one query of every accumulator each, so four
+//   warps 2-25  epilogue: TMEM -> registers, ReLU, weighted head sum, store.
+//               Six sets of four warps (one warp per TMEM lane quadrant in
+//               each) take the (accumulator, query) units in turn, so six
 //               warps per SM sub-partition hide each other's latencies.  A
 //               score costs per head one max (the ReLU) and half of a packed
 //               two-lane fp32 FMA, into four independent accumulator pairs.
@@ -44,6 +44,12 @@ constexpr int kHI = 64, kDI = 128, kTileK = 128;  // heads, dims, keys per tile
 constexpr int kThreads = 576;
 constexpr int kEpiThreads = 512;  // warps 2-17
 constexpr int kEpiSets = kEpiThreads / 128;
+// Prefill: six sets of four epilogue warps (warps 2-25) share out the
+// (accumulator, query) units in turn; the extra warps hide the latency of
+// each unit's TMEM loads and weight reads behind the others' arithmetic.
+constexpr int kEpiSetsP = 6;
+constexpr int kEpiThreadsP = kEpiSetsP * 128;  // 768
+constexpr int kThreadsP = 64 + kEpiThreadsP;   // 832
 
 // Two fp32 FMAs in one instruction: {lo, hi} = {x0 * w0, x1 * w1} + acc.
 __device__ __forceinline__ uint64_t fma2(float x0, float x1, float w0, float w1, uint64_t acc) {
@@ -164,7 +170,7 @@ __device__ Work plan_prefill(const Rows& R, int32_t row0, int32_t nrows) {
 }
 
 template <int DT, int G, int NG, int NK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsP, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ CUtensorMap kmap, Rows R, int32_t row0,
                       int32_t nrows, const float* __restrict__ w, const float* __restrict__ q_scale,
@@ -197,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < C::NS; ++i) {
       mbar_init(s_full(i), 1);
-      mbar_init(s_empty(i), kEpiThreads / 32);  // every epilogue warp
+      mbar_init(s_empty(i), 4 * G);  // the four lane-quadrant warps of each of the G queries
     }
     mbar_init(q_full, 1);
     mbar_init(drain, 1);
@@ -288,10 +294,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int et = tid - 64;           // 0..511
+    const int et = tid - 64;           // 0..767
     const int quad = warp & 3;         // TMEM lane quadrant this warp may read
-    const int set = et >> 7;           // warps 2-5: set 0, 6-9: set 1, ...
-    for (int i = et; i < C::QB * kHI; i += kEpiThreads) {
+    const int set = et >> 7;           // warps 2-5: set 0, 6-9: set 1, ... 22-25: set 5
+    for (int i = et; i < C::QB * kHI; i += kEpiThreadsP) {
       const int qi = i / kHI, h = i - qi * kHI;
       const int32_t tq = wk.t0 + qi;
       float v = 0.f;
@@ -302,53 +308,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       wq[i] = v;
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
-    // queries of each accumulator this set handles
-    static_assert(G % kEpiSets == 0, "every epilogue set takes a share of each accumulator");
-    constexpr int QS = G / kEpiSets;
-    // the key scale of this thread's key, loaded one tile ahead
-    auto key_scale = [&](int j) {
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreadsP) : "memory");
+    // Unit u = (accumulator u / G, query u % G); set `set` takes units set,
+    // set + 6, ...  G < 6, so a set reads each accumulator at most once.
+    static_assert(G < kEpiSetsP, "one unit of an accumulator per set");
+    const int n_units = n_tiles * NG * G;
+    for (int u = set; u < n_units; u += kEpiSetsP) {
+      const int job = u / G, qq = u - job * G;
+      const int j = job / NG, g = job - j * NG;
+      const int slot = job % C::NS;
       const int32_t s = (wk.kt_begin + j) * kTileK + quad * 32 + lane;
-      return (DT == DSA_E4M3 && k_scale && j < n_tiles && s < wk.len) ? __ldg(k_scale + wk.kbase + s)
-                                                                      : 1.f;
-    };
-    float ks_next = key_scale(0);
-    int job = 0;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int32_t s = (wk.kt_begin + j) * kTileK + quad * 32 + lane;
-      const float ks = ks_next;
-      ks_next = key_scale(j + 1);
-      for (int g = 0; g < NG; ++g, ++job) {
-        const int slot = job % C::NS;
-        // warp-uniform: the tcgen05 loads below need the whole warp
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(s_full(slot), (job / C::NS) & 1, R.status) && !*abort_flag)) {
-          *abort_flag = 1;
-          j = n_tiles;
-          break;
+      // the key scale is fetched before the wait, which hides its latency
+      const float ks = (DT == DSA_E4M3 && k_scale && s < wk.len) ? __ldg(k_scale + wk.kbase + s) : 1.f;
+      // warp-uniform: the tcgen05 loads below need the whole warp
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(s_full(slot), (job / C::NS) & 1, R.status) && !*abort_flag)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int qi = g * G + qq;
+      const float4* wr = reinterpret_cast<const float4*>(wq + qi * kHI);
+      const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + slot * C::N + qq * kHI;
+      uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float v[32];
+        tmem_ld32(ta + 32 * half, v);
+#pragma unroll
+        for (int h4 = 0; h4 < 8; ++h4) {
+          const float4 w4 = wr[8 * half + h4];
+          acc[(2 * h4) & 3] = fma2(fmaxf(v[4 * h4], 0.f), fmaxf(v[4 * h4 + 1], 0.f), w4.x, w4.y,
+                                   acc[(2 * h4) & 3]);
+          acc[(2 * h4 + 1) & 3] = fma2(fmaxf(v[4 * h4 + 2], 0.f), fmaxf(v[4 * h4 + 3], 0.f),
+                                       w4.z, w4.w, acc[(2 * h4 + 1) & 3]);
         }
-        tc_fence_after();
-        {
-#pragma unroll 1
-          for (int qs = 0; qs < QS; ++qs) {
-            const int qq = set * QS + qs;
-            const int qi = g * G + qq;
-            const float4* wr = reinterpret_cast<const float4*>(wq + qi * kHI);
-            const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + slot * C::N + qq * kHI;
-            const float sum = relu_wsum(ta, wr);
-            const int32_t tq = wk.t0 + qi;
-            if (tq >= wk.qvalid_lo && tq < wk.qvalid_hi && s < R.max_len) {
-              float* o = scores + (int64_t)(wk.qrow0 + qi - row0) * ld;
-              if (s <= tq)
-                o[s] = sum * ks;
-              else if (fill)
-                o[s] = -INFINITY;
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_empty(slot));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_empty(slot));
+      const float sum = (lo32(acc[0]) + hi32(acc[0])) + (lo32(acc[1]) + hi32(acc[1])) +
+                        ((lo32(acc[2]) + hi32(acc[2])) + (lo32(acc[3]) + hi32(acc[3])));
+      const int32_t tq = wk.t0 + qi;
+      if (tq >= wk.qvalid_lo && tq < wk.qvalid_hi && s < R.max_len) {
+        float* o = scores + (int64_t)(wk.qrow0 + qi - row0) * ld;
+        if (s <= tq)
+          o[s] = sum * ks;
+        else if (fill)
+          o[s] = -INFINITY;
       }
     }
     // -inf beyond the last scored tile (unit call only)
@@ -358,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (qi >= wk.nq || tq < wk.qvalid_lo || tq >= wk.qvalid_hi) continue;
         float* o = scores + (int64_t)(wk.qrow0 + qi - row0) * ld;
         const int32_t from = wk.kt_end * kTileK;
-        for (int s = from + et; s < R.max_len; s += kEpiThreads) o[s] = -INFINITY;
+        for (int s = from + et; s < R.max_len; s += kEpiThreadsP) o[s] = -INFINITY;
       }
     }
   }
@@ -769,7 +776,7 @@ static dsa_status_t launch_cfg(const Rows& R, int32_t row0, int32_t nrows, const
     return DSA_ERR_CUDA;
   const int32_t span = nrows < R.max_len ? nrows : R.max_len;
   const dim3 grid((span + C::QB - 1) / C::QB + 1, R.B);
-  kfn<<<grid, kThreads, C::SMEM, st>>>(qmap, kmap, R, row0, nrows, w, q_scale, k_scale, scores,
+  kfn<<<grid, kThreadsP, C::SMEM, st>>>(qmap, kmap, R, row0, nrows, w, q_scale, k_scale, scores,
                                        ld, fill ? 1 : 0);
   return launch_status();
 }
