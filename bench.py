@@ -1,7 +1,7 @@
 """Throughput of the DSA hot path (indexer -> top-k -> sparse MLA attention).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dsa|reference]
-                    [--workload prefill64k|decode64k|prefill8k|decode128k|tiny]
+                    [--workload prefill64k|decode64k|prefill8k|decode128k|chunked64k|tiny]
 
 One JSON line on rank 0.  A step is one dsa_forward over the whole workload
 (every stage of the path).  The default workload is the 64K-token prefill
@@ -45,7 +45,7 @@ import workloads  # noqa: E402
 METRIC = "DSA prefill & decode tokens/s at 64K ctx, k=2048; % of TC/HBM roofline"
 
 WORKLOADS = {
-    "tiny": 1, "prefill8k": 2, "decode64k": 3, "prefill64k": 4, "decode128k": 5,
+    "tiny": 1, "prefill8k": 2, "decode64k": 3, "prefill64k": 4, "decode128k": 5, "chunked64k": 6,
 }
 DESCR = {
     1: "DSA prefill, 1 x 256 tokens, fp32 indexer 4x32, k=32, MLA 8 heads 80/64 bf16",
@@ -56,6 +56,8 @@ DESCR = {
        "MLA 128 heads 576/512 bf16",
     5: "DSA decode, 16 sequences x 1 query, cache 131072, e4m3 indexer, k=2048, MLA 128 heads "
        "576/512 bf16",
+    6: "DSA chunked prefill, 4 sequences x 65536 cached tokens, the last 4096 of each new "
+       "(16384 query rows), e4m3 indexer 64x128, k=2048, MLA 128 heads 576/512 bf16",
 }
 
 
@@ -169,7 +171,7 @@ def run_device(cid, steps, warmup, rank, world, do_e2e=True):
     wl = workloads.generate(cid, pin=do_e2e)
     c = wl.cfg
     d = wl.to(dev)
-    lay = dsa.Layout.of(wl, d.kv_offsets)
+    lay = dsa.Layout.of(wl, d.kv_offsets, d.q_offsets)
     args = dsa.forward_args(q_idx=d.q_idx, q_scale=d.q_scale, w=d.w, k_idx=d.k_idx,
                             k_scale=d.k_scale, q=d.q, kv=d.kv, D_V=c.D_V, sm_scale=c.sm_scale,
                             k=c.k)
@@ -232,20 +234,25 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
     the step's inputs from pinned host memory and reads the result back.
 
     Prefill: the step's inputs are the whole sequence (queries, indexer keys,
-    MLA cache), all copied every step.  Decode: the caches are state that
-    earlier steps built and that stays in HBM (copied once, untimed); a step's
-    inputs are the new queries and each sequence's newest cache row (indexer
-    key, its scale, latent + rotary row), appended in place every step."""
-    names = ["q_idx", "q_scale", "w", "k_idx", "k_scale", "q", "kv", "kv_offsets"]
-    cache = ("k_idx", "k_scale", "kv") if c.mode == "decode" else ()
+    MLA cache), all copied every step.  Decode and chunked prefill: the caches
+    are state that earlier steps built and that stays in HBM (copied once,
+    untimed); a step's inputs are the new queries and the cache rows of the
+    new tokens (indexer key, its scale, latent + rotary row: one per sequence
+    in decode, the chunk's in chunked prefill), written in place every step."""
+    names = ["q_idx", "q_scale", "w", "k_idx", "k_scale", "q", "kv", "kv_offsets", "q_offsets"]
+    resident = c.mode in ("decode", "chunked")
+    cache = ("k_idx", "k_scale", "kv") if resident else ()
     host = {n: getattr(wl, n) for n in names if getattr(wl, n) is not None}
     dbuf = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
-    for n in cache + ("kv_offsets",) if c.mode == "decode" else ():
+    for n in cache + ("kv_offsets", "q_offsets") if resident else ():
         if n in host:
             dbuf[n].copy_(host.pop(n))  # resident state, outside the timed region
     new_rows = {}
     if cache:
-        last = torch.from_numpy(wl.kv_offsets.numpy()[1:].astype("int64") - 1)
+        ends = wl.kv_offsets.numpy()[1:].astype("int64")
+        fresh = [1] * wl.B if c.mode == "decode" else list(c.chunks)
+        last = torch.from_numpy(np.concatenate(
+            [np.arange(e - f, e) for e, f in zip(ends, fresh)]).astype("int64"))
         last_dev = last.to(dev)
         for n in cache:
             if n in dbuf:
@@ -258,7 +265,7 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
     out_h = torch.empty(wl.n_q, c.H, c.D_V, dtype=torch.bfloat16, pin_memory=True)
     lse_h = torch.empty(wl.n_q, c.H, dtype=torch.float32, pin_memory=True)
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
-    lay2 = dsa.Layout.of(wl, dbuf["kv_offsets"])
+    lay2 = dsa.Layout.of(wl, dbuf["kv_offsets"], dbuf.get("q_offsets"))
     args = dsa.forward_args(q_idx=dbuf["q_idx"], q_scale=dbuf.get("q_scale"), w=dbuf["w"],
                             k_idx=dbuf["k_idx"], k_scale=dbuf.get("k_scale"), q=dbuf["q"],
                             kv=dbuf["kv"], D_V=c.D_V, sm_scale=c.sm_scale, k=c.k)
@@ -268,9 +275,12 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
     def one():
         for n, t in host.items():
             dbuf[n].copy_(t, non_blocking=True)
-        for n, (h, stage) in new_rows.items():  # decode: append the newest cache rows
+        for n, (h, stage) in new_rows.items():  # the new tokens' cache rows, in place
             stage.copy_(h, non_blocking=True)
-            dbuf[n].index_copy_(0, last_dev, stage)
+            if stage.dtype == torch.float8_e4m3fn:  # no fp8 index_copy: move the bytes
+                dbuf[n].view(torch.uint8).index_copy_(0, last_dev, stage.view(torch.uint8))
+            else:
+                dbuf[n].index_copy_(0, last_dev, stage)
         dsa.dsa_forward(lay2, args, out, lse, None, ws)
         out_h.copy_(out, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
@@ -284,7 +294,7 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
     e1.record(stream)
     e1.synchronize()
     ms = e0.elapsed_time(e1) / steps
-    inputs = ("new queries + each sequence's newest cache row per step (caches resident in HBM)"
+    inputs = ("new queries + the new tokens' cache rows per step (caches resident in HBM)"
               if cache else "every input of the step (queries, indexer keys, MLA cache)")
     return {"ms_per_step": ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "inputs": inputs}

@@ -49,7 +49,7 @@ typedef enum {
 
 typedef enum { DSA_F32 = 0, DSA_BF16 = 1, DSA_E4M3 = 2 } dsa_dtype_t;
 
-typedef enum { DSA_PREFILL = 0, DSA_DECODE = 1 } dsa_mode_t;
+typedef enum { DSA_PREFILL = 0, DSA_DECODE = 1, DSA_CHUNKED = 2 } dsa_mode_t;
 
 /*
  * Ragged layout shared by every call.
@@ -62,6 +62,14 @@ typedef enum { DSA_PREFILL = 0, DSA_DECODE = 1 } dsa_mode_t;
  *    t = r - kv_offsets[b] and sees positions 0..t.
  *  - DECODE: one query per sequence, n_q == B; query row b sits at position
  *    t = L_b - 1 (the cache already holds the new token) and sees 0..t.
+ *  - CHUNKED: a prefill of new tokens against a cache that already holds
+ *    earlier ones (chunked prefill with a prefix cache).  Sequence b owns
+ *    query rows q_offsets[b] .. q_offsets[b+1]-1, C_b of them, its LAST C_b
+ *    positions: query i sits at t = L_b - C_b + i and sees 0..t (the cache
+ *    already holds the chunk's own tokens).  n_q == q_offsets[B].  PREFILL is
+ *    the case C_b = L_b, DECODE the case C_b = 1.  q_offsets must be
+ *    non-decreasing with C_b <= L_b; a sequence that breaks this is skipped
+ *    on the device and reported as DSA_ERR_DEVICE_DATA.
  * The candidate set of a query is s <= t, the causal lower triangle
  * ("GLM sparse attention", 56-token causal figure; the diagonal included).
  */
@@ -72,6 +80,7 @@ typedef struct {
   int32_t max_len;           /* >= every L_b; the row stride of score arrays */
   int32_t n_q;               /* query rows (see above) */
   int64_t n_k;               /* cache rows = kv_offsets[B] */
+  const int32_t* q_offsets;  /* CHUNKED only: DEVICE [B+1], q_offsets[0] = 0; else unused */
 } dsa_layout_t;
 
 /*

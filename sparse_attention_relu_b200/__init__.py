@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_HERE, "libdsa.so")
 DSA_OK, DSA_ERR_INVALID_ARGUMENT, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE = 0, 1, 2, 3
 DSA_ERR_CUDA, DSA_ERR_TIMEOUT, DSA_ERR_DEVICE_DATA = 4, 5, 6
 DSA_F32, DSA_BF16, DSA_E4M3 = 0, 1, 2
-DSA_PREFILL, DSA_DECODE = 0, 1
+DSA_PREFILL, DSA_DECODE, DSA_CHUNKED = 0, 1, 2
 
 _DTYPE_CODE = {torch.float32: DSA_F32, torch.bfloat16: DSA_BF16, torch.float8_e4m3fn: DSA_E4M3}
 
@@ -38,7 +38,8 @@ class DSAError(RuntimeError):
 class dsa_layout_t(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("batch", ctypes.c_int32),
                 ("kv_offsets", ctypes.c_void_p), ("max_len", ctypes.c_int32),
-                ("n_q", ctypes.c_int32), ("n_k", ctypes.c_int64)]
+                ("n_q", ctypes.c_int32), ("n_k", ctypes.c_int64),
+                ("q_offsets", ctypes.c_void_p)]
 
 
 class dsa_forward_args_t(ctypes.Structure):
@@ -123,16 +124,21 @@ def _check(status: int, where: str):
 class Layout:
     """The ragged layout of include/dsa.h, built from a device int32 offsets tensor."""
 
-    def __init__(self, kv_offsets: torch.Tensor, mode: int, max_len: int, n_q: int, n_k: int):
-        self.kv_offsets = kv_offsets  # keeps the tensor alive
+    def __init__(self, kv_offsets: torch.Tensor, mode: int, max_len: int, n_q: int, n_k: int,
+                 q_offsets: torch.Tensor = None):
+        self.kv_offsets = kv_offsets  # keeps the tensors alive
+        self.q_offsets = q_offsets
         self.c = dsa_layout_t(int(mode), int(kv_offsets.numel() - 1), _ptr(kv_offsets),
-                              int(max_len), int(n_q), int(n_k))
+                              int(max_len), int(n_q), int(n_k), _ptr(q_offsets))
 
     @classmethod
-    def of(cls, wl, kv_offsets: torch.Tensor):
-        """Layout of a workloads.Workload whose offsets already sit on the device."""
-        mode = DSA_PREFILL if wl.cfg.mode == "prefill" else DSA_DECODE
-        return cls(kv_offsets, mode, wl.max_len, wl.n_q, wl.n_k)
+    def of(cls, wl, kv_offsets: torch.Tensor, q_offsets: torch.Tensor = None):
+        """Layout of a workloads.Workload whose offsets already sit on the device
+        (q_offsets: the chunked mode's query offsets, on the device too)."""
+        mode = {"prefill": DSA_PREFILL, "decode": DSA_DECODE, "chunked": DSA_CHUNKED}[wl.cfg.mode]
+        if mode == DSA_CHUNKED and q_offsets is None:
+            raise ValueError("chunked layout needs the device q_offsets")
+        return cls(kv_offsets, mode, wl.max_len, wl.n_q, wl.n_k, q_offsets)
 
     @property
     def ref(self):

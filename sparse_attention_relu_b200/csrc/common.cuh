@@ -21,6 +21,7 @@ enum : unsigned {
 struct Rows {
   unsigned* status;     // this device's status word (see dsa_device_status)
   const int32_t* offs;  // [B+1] device
+  const int32_t* qoffs;  // [B+1] device, CHUNKED only (query rows of each sequence)
   int32_t B;
   int32_t mode;  // DSA_PREFILL / DSA_DECODE
   int32_t max_len;
@@ -43,6 +44,26 @@ struct RowInfo {
 // empty (t = -1) and raise kErrBadOffsets.
 __device__ __forceinline__ RowInfo row_info(const Rows& R, int32_t r) {
   RowInfo ri{0, -1, 0, 0};
+  if (R.mode == DSA_CHUNKED) {
+    // largest b with qoffs[b] <= r; query i of b sits at L_b - C_b + i
+    int32_t lo = 0, hi = R.B - 1;
+    while (lo < hi) {
+      int32_t mid = (lo + hi + 1) >> 1;
+      if (__ldg(R.qoffs + mid) <= r) lo = mid; else hi = mid - 1;
+    }
+    const int32_t q0 = __ldg(R.qoffs + lo), q1 = __ldg(R.qoffs + lo + 1);
+    const int32_t o0 = __ldg(R.offs + lo), o1 = __ldg(R.offs + lo + 1);
+    if (q0 < 0 || q1 < q0 || r < q0 || r >= q1 || q1 > R.n_q || o0 < 0 || o1 < o0 ||
+        (int64_t)o1 > R.n_k || o1 - o0 > R.max_len || q1 - q0 > o1 - o0) {
+      raise_status(R, kErrBadOffsets);
+      return ri;
+    }
+    ri.kbase = o0;
+    ri.len = o1 - o0;
+    ri.t = ri.len - (q1 - q0) + (r - q0);
+    ri.seq = lo;
+    return ri;
+  }
   if (R.mode == DSA_DECODE) {
     int32_t b = r;
     int32_t o0 = __ldg(R.offs + b), o1 = __ldg(R.offs + b + 1);

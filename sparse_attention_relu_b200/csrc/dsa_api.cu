@@ -40,19 +40,25 @@ __global__ void wait_timeout_selftest(unsigned* status, long long limit) {
 // Checks the layout; fills the device-side row description.
 dsa_status_t check_layout(const dsa_layout_t* L, Rows* R) {
   if (!L) return DSA_ERR_INVALID_ARGUMENT;
-  if (L->mode != DSA_PREFILL && L->mode != DSA_DECODE) return DSA_ERR_INVALID_ARGUMENT;
+  if (L->mode != DSA_PREFILL && L->mode != DSA_DECODE && L->mode != DSA_CHUNKED)
+    return DSA_ERR_INVALID_ARGUMENT;
   if (L->batch < 0 || L->max_len < 0 || L->n_q < 0 || L->n_k < 0) return DSA_ERR_INVALID_ARGUMENT;
   if (L->batch > 0 && (!L->kv_offsets || !aligned16(L->kv_offsets)))
     return DSA_ERR_INVALID_ARGUMENT;
   if (L->n_k >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;  // int32 offsets
   if (L->mode == DSA_PREFILL) {
     if (L->n_q != L->n_k) return DSA_ERR_INVALID_ARGUMENT;
-  } else {
+  } else if (L->mode == DSA_DECODE) {
     if (L->n_q != L->batch) return DSA_ERR_INVALID_ARGUMENT;
+  } else {  // CHUNKED: every query is a cache row of its sequence
+    if (L->batch > 0 && (!L->q_offsets || !aligned16(L->q_offsets)))
+      return DSA_ERR_INVALID_ARGUMENT;
+    if ((int64_t)L->n_q > L->n_k) return DSA_ERR_INVALID_ARGUMENT;
   }
   if (L->n_q > 0 && (L->batch == 0 || L->max_len == 0)) return DSA_ERR_INVALID_ARGUMENT;
   R->status = nullptr;  // filled by device_rows() once every argument passed
   R->offs = L->kv_offsets;
+  R->qoffs = L->mode == DSA_CHUNKED ? L->q_offsets : nullptr;
   R->B = L->batch;
   R->mode = L->mode;
   R->max_len = L->max_len;
@@ -169,7 +175,7 @@ using namespace dsa;
 
 extern "C" {
 
-int32_t dsa_abi_version(void) { return 1; }
+int32_t dsa_abi_version(void) { return 2; }
 
 const char* dsa_status_string(dsa_status_t s) {
   switch (s) {

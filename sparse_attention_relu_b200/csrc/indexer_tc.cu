@@ -142,27 +142,38 @@ struct Work {
   int32_t qvalid_lo, qvalid_hi;  // valid query positions [lo, hi) (local)
 };
 
+// PREFILL and CHUNKED: a block owns QB consecutive query rows of sequence
+// blockIdx.y.  In PREFILL a sequence's query rows are its cache rows
+// (positions 0 ..); in CHUNKED they are q_offsets[b] .. q_offsets[b+1]-1 at
+// the last C_b positions (the first at p0 = L_b - C_b).
 template <int QB>
 __device__ Work plan_prefill(const Rows& R, int32_t row0, int32_t nrows) {
   Work w{};
   const int b = blockIdx.y;
   const int32_t o0 = __ldg(R.offs + b), o1 = __ldg(R.offs + b + 1);
-  if (o0 < 0 || o1 < o0 || (int64_t)o1 > R.n_k || o1 - o0 > R.max_len) {
+  int32_t q0 = o0, q1 = o1;
+  if (R.mode == DSA_CHUNKED) {
+    q0 = __ldg(R.qoffs + b);
+    q1 = __ldg(R.qoffs + b + 1);
+  }
+  if (o0 < 0 || o1 < o0 || (int64_t)o1 > R.n_k || o1 - o0 > R.max_len || q0 < 0 || q1 < q0 ||
+      q1 > R.n_q || q1 - q0 > o1 - o0) {
     if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(R, kErrBadOffsets);
     return w;
   }
-  const int32_t lo = max(o0, row0), hi = min(o1, row0 + nrows);
+  const int32_t p0 = (o1 - o0) - (q1 - q0);  // position of the sequence's first query
+  const int32_t lo = max(q0, row0), hi = min(q1, row0 + nrows);
   if (lo >= hi) return w;
-  const int32_t i0 = (lo - o0) / QB, i1 = (hi - 1 - o0) / QB;
+  const int32_t i0 = (lo - q0) / QB, i1 = (hi - 1 - q0) / QB;
   if ((int32_t)blockIdx.x > i1 - i0) return w;
   const int32_t i = i1 - (int32_t)blockIdx.x;  // heaviest block first
   w.valid = 1;
   w.kbase = o0;
   w.len = o1 - o0;
-  w.t0 = i * QB;
-  w.qrow0 = o0 + w.t0;
-  w.qvalid_lo = max(w.t0, lo - o0);
-  w.qvalid_hi = min(w.t0 + QB, hi - o0);
+  w.t0 = p0 + i * QB;
+  w.qrow0 = q0 + i * QB;
+  w.qvalid_lo = p0 + max(i * QB, lo - q0);
+  w.qvalid_hi = p0 + min(i * QB + QB, hi - q0);
   w.nq = QB;
   w.kt_begin = 0;
   w.kt_end = (w.qvalid_hi - 1) / kTileK + 1;  // keys up to the last valid query

@@ -82,7 +82,7 @@ def indexer_topk(stage: str, reps: int, T: int, k: int = 2048):
     cfg = workloads.custom("prefill", [T], idx_dtype="e4m3", k=k)
     wl = workloads.generate(cfg, with_mla=False)
     d = wl.to("cuda")
-    lay = dsa.Layout.of(wl, d.kv_offsets)
+    lay = dsa.Layout.of(wl, d.kv_offsets, d.q_offsets)
     scores = torch.empty(T, T, dtype=torch.float32, device="cuda")
     idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
     ind = lambda: dsa.dsa_indexer_scores(lay, d.q_idx, d.q_scale, d.w, d.k_idx, d.k_scale, scores)

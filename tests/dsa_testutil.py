@@ -26,7 +26,7 @@ class Dev:
         self.wl = wl
         d = wl.to("cuda")
         self.d = d
-        self.layout = dsa.Layout.of(wl, d.kv_offsets)
+        self.layout = dsa.Layout.of(wl, d.kv_offsets, d.q_offsets)
         torch.cuda.synchronize()
 
     def scores(self):

@@ -19,7 +19,7 @@ from dsa_testutil import (Dev, assert_attn_close, assert_scores_close, assert_se
 
 pytestmark = pytest.mark.gpu
 
-SAMPLES = {1: None, 2: 12, 3: 8, 4: 8, 5: 4}
+SAMPLES = {1: None, 2: 12, 3: 8, 4: 8, 5: 4, 6: 8}
 
 
 def _rows(wl, n):
@@ -31,7 +31,7 @@ def _rows(wl, n):
     return workloads.sample_rows(wl.n_q, n, must)
 
 
-@pytest.mark.parametrize("cid", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("cid", [1, 2, 3, 4, 5, 6])
 def test_forward_matches_oracle(cid):
     wl = workloads.generate(cid)
     dev = Dev(wl)

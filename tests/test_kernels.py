@@ -30,6 +30,12 @@ SMALL = {
     # range crossing several rows, runs of one-tile rows among them
     "decode_bf16_many_rows": workloads.custom("decode", _MANY, idx_dtype="bf16", k=64),
     "decode_e4m3_many_rows": workloads.custom("decode", _MANY[::-1], idx_dtype="e4m3", k=96),
+    # chunked prefill against a prefix cache: the last C_b positions of each
+    # sequence are new queries (a whole sequence, and one-token chunks, included)
+    "chunked_bf16": workloads.custom("chunked", [700, 300, 2049, 129], idx_dtype="bf16", k=128,
+                                     chunks=[100, 300, 37, 1]),
+    "chunked_e4m3": workloads.custom("chunked", [3000, 130], idx_dtype="e4m3", k=256,
+                                     chunks=[260, 130]),
     "prefill_f32_generic_dims": workloads.custom("prefill", [150], H_I=16, D_I=64,
                                                  idx_dtype="f32", k=20, H=20, D_K=96, D_V=32),
 }
@@ -174,3 +180,36 @@ def test_index_order_does_not_matter():
     o2, l2 = dev.attn(perm)
     assert (o1.float() - o2.float()).abs().max().item() <= 2e-3
     assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+def _scores_of(cfg):
+    dev = Dev(workloads.generate(cfg))
+    return dev, dev.scores()
+
+
+def test_chunked_reduces_to_prefill_and_decode():
+    """A chunk that is the whole sequence is a prefill; one-token chunks are a
+    decode step.  Same seeded data, same scores (the prefill form runs the
+    same kernel, so exactly; the decode form runs the decode kernel, so to
+    rounding), and the same attention output on the same indices."""
+    lens = [900, 333, 1500]
+    pre_dev, pre = _scores_of(workloads.custom("prefill", lens, k=128, seed=21))
+    ch_dev, ch = _scores_of(workloads.custom("chunked", lens, k=128, seed=21, chunks=lens))
+    assert dsa.dsa_device_status() == dsa.DSA_OK
+    assert torch.equal(torch.nan_to_num(ch, neginf=-1e30), torch.nan_to_num(pre, neginf=-1e30))
+    idx = pre_dev.topk(pre)
+    o_pre, l_pre = pre_dev.attn(idx)
+    o_ch, l_ch = ch_dev.attn(idx)
+    assert torch.equal(o_pre, o_ch) and torch.equal(l_pre, l_ch)
+
+    dec_dev, dec = _scores_of(workloads.custom("decode", lens, k=128, seed=22))
+    one_dev, one = _scores_of(workloads.custom("chunked", lens, k=128, seed=22,
+                                               chunks=[1] * len(lens)))
+    assert dsa.dsa_device_status() == dsa.DSA_OK
+    fin = torch.isfinite(dec)
+    assert torch.equal(fin, torch.isfinite(one))
+    assert torch.allclose(one[fin], dec[fin], rtol=1e-5, atol=1e-6)
+    idx = dec_dev.topk(dec)
+    o_dec, l_dec = dec_dev.attn(idx)
+    o_one, l_one = one_dev.attn(idx)
+    assert torch.equal(o_dec, o_one) and torch.equal(l_dec, l_one)

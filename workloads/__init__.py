@@ -40,7 +40,7 @@ E4M3_MAX = 448.0
 class Config:
     cid: int
     name: str
-    mode: str  # "prefill" | "decode"
+    mode: str  # "prefill" | "decode" | "chunked"
     lens: Optional[List[int]]  # per-sequence cache lengths (None: drawn, see len_range)
     B: int
     H_I: int
@@ -57,6 +57,7 @@ class Config:
     len_range: Optional[tuple] = None
     alpha: float = 64.0
     seed: int = 0
+    chunks: Optional[List[int]] = None  # chunked: new query tokens per sequence (<= its length)
 
     def __post_init__(self):
         if not self.seed:
@@ -64,7 +65,8 @@ class Config:
 
 
 def config(cid: int) -> Config:
-    """The five workloads, by number (1 = tiny prefill ... 5 = 128K decode)."""
+    """The five workloads, by number (1 = tiny prefill ... 5 = 128K decode), and 6: a
+    chunked prefill against a prefix cache (beyond the five, for that mode)."""
     if cid == 1:
         return Config(1, "prefill_T256_tiny_f32", "prefill", [256], 1, 4, 32, "f32", 32, 8, 80,
                       64, 1 / math.sqrt(80), math.sqrt(1 / 4), 1 / math.sqrt(80))
@@ -83,19 +85,27 @@ def config(cid: int) -> Config:
         return Config(5, "decode_B16_L131072_e4m3_sinks", "decode", [131072] * 16, 16, 64, 128,
                       "e4m3", 2048, 128, 576, 512, 1 / math.sqrt(576), math.sqrt(1 / 64),
                       1 / math.sqrt(576), plant="sinks_window")
+    if cid == 6:
+        # chunked prefill with a prefix cache: 4 sequences of 65,536 cached tokens,
+        # the last 4,096 of each new (16,384 query rows); e4m3 indexer as config 4
+        return Config(6, "chunked_B4_L65536_C4096_e4m3", "chunked", [65536] * 4, 4, 64, 128,
+                      "e4m3", 2048, 128, 576, 512, 1 / math.sqrt(576), math.sqrt(1 / 64),
+                      1 / math.sqrt(576), chunks=[4096] * 4)
     raise ValueError(f"unknown config {cid}")
 
 
 def custom(mode="prefill", lens=(300,), H_I=64, D_I=128, idx_dtype="bf16", k=64, H=128,
            D_K=576, D_V=512, sm_scale=None, w_std=None, mla_std=None, plant=None, seed=7,
-           name=None) -> Config:
-    """A small workload with the structure of the big ones (tests)."""
+           name=None, chunks=None) -> Config:
+    """A small workload with the structure of the big ones (tests).  For
+    mode "chunked", chunks[b] new query tokens close sequence b."""
     lens = list(lens)
     return Config(0, name or f"custom_{mode}_{idx_dtype}", mode, lens, len(lens), H_I, D_I,
                   idx_dtype, k, H, D_K, D_V,
                   sm_scale if sm_scale is not None else 1 / math.sqrt(D_K),
                   w_std if w_std is not None else 1 / math.sqrt(H_I),
-                  mla_std if mla_std is not None else 1 / math.sqrt(D_K), plant=plant, seed=seed)
+                  mla_std if mla_std is not None else 1 / math.sqrt(D_K), plant=plant, seed=seed,
+                  chunks=list(chunks) if chunks is not None else None)
 
 
 def _seed(*parts) -> int:
@@ -156,10 +166,20 @@ class Workload:
         offs[1:] = np.cumsum(lens)
         self.kv_offsets = torch.from_numpy(offs.astype(np.int32))
         self.n_k = int(offs[-1])
+        self.q_offsets = None
         if cfg.mode == "prefill":
             self.seq = np.repeat(np.arange(self.B), lens).astype(np.int64)
             self.tpos = np.concatenate([np.arange(L) for L in lens]).astype(np.int64) \
                 if self.B else np.zeros(0, np.int64)
+        elif cfg.mode == "chunked":
+            chunks = list(cfg.chunks)
+            assert len(chunks) == self.B and all(0 <= c <= L for c, L in zip(chunks, lens))
+            self.seq = np.repeat(np.arange(self.B), chunks).astype(np.int64)
+            self.tpos = np.concatenate([np.arange(L - c, L) for L, c in zip(lens, chunks)]) \
+                .astype(np.int64) if self.B else np.zeros(0, np.int64)
+            qo = np.zeros(self.B + 1, np.int64)
+            qo[1:] = np.cumsum(chunks)
+            self.q_offsets = torch.from_numpy(qo.astype(np.int32))
         else:
             self.seq = np.arange(self.B, dtype=np.int64)
             self.tpos = np.array([L - 1 for L in lens], np.int64)
@@ -188,7 +208,7 @@ class Workload:
             raise ValueError(cfg.idx_dtype)
         del qI, kI
         if pin:
-            for name in ("q_idx", "k_idx", "w", "q_scale", "k_scale", "kv_offsets"):
+            for name in ("q_idx", "k_idx", "w", "q_scale", "k_scale", "kv_offsets", "q_offsets"):
                 t = getattr(self, name)
                 if t is not None:
                     setattr(self, name, t.pin_memory())
@@ -245,7 +265,8 @@ class Workload:
         """A shallow copy whose tensors live on ``device``."""
         other = object.__new__(Workload)
         other.__dict__.update(self.__dict__)
-        for name in ("q_idx", "k_idx", "w", "q_scale", "k_scale", "kv_offsets", "q", "kv"):
+        for name in ("q_idx", "k_idx", "w", "q_scale", "k_scale", "kv_offsets", "q_offsets", "q",
+                     "kv"):
             t = getattr(self, name)
             if t is not None:
                 setattr(other, name, t.to(device, non_blocking=True))
