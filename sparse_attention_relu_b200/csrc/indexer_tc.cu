@@ -700,14 +700,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const RowInfo ri = row_info(R, row0 + sg.r);
       const float4* wr = reinterpret_cast<const float4*>(wq + qb * kHI);
       float* o = scores + (int64_t)sg.r * ld;
-      for (int j = sg.kb; j < sg.ke; ++j, ++gt) {
-        if ((int)(gt % kEpiSets) != set) continue;
-        const int slot = (int)(gt % C::NS);
+      // this set's accumulators in the segment: tiles j0, j0 + 4, ...; the key
+      // scales of the next one are fetched while this one is summed (the MMAs
+      // run ahead, so the scale load would otherwise stand alone in the way)
+      const int64_t gt0 = gt;
+      const int j0 = sg.kb + (int)((set - (int)(gt0 % kEpiSets) + kEpiSets) % kEpiSets);
+      auto key_scale = [&](int j) {
         const int32_t s = j * kTileK + quad * 32 + lane;
-        float ks = 1.f;
-        if (DT == DSA_E4M3 && k_scale && s <= ri.t) ks = __ldg(k_scale + ri.kbase + s);
+        return (DT == DSA_E4M3 && k_scale && j < sg.ke && s <= ri.t) ? __ldg(k_scale + ri.kbase + s)
+                                                                     : 1.f;
+      };
+      float ks_next = key_scale(j0);
+      gt = gt0 + (sg.ke - sg.kb);
+      for (int j = j0; j < sg.ke; j += kEpiSets) {
+        const int64_t gj = gt0 + (j - sg.kb);
+        const int slot = (int)(gj % C::NS);
+        const int32_t s = j * kTileK + quad * 32 + lane;
+        const float ks = ks_next;
+        ks_next = key_scale(j + kEpiSets);
         if (!__all_sync(0xffffffffu,
-                        mbar_wait(s_full(slot), (int)((gt / C::NS) & 1), R.status) && !*abort_flag)) {
+                        mbar_wait(s_full(slot), (int)((gj / C::NS) & 1), R.status) && !*abort_flag)) {
           ok = false;
           break;
         }
