@@ -13,7 +13,10 @@ Timing: W untimed warm-up steps, then K steps, each preceded by an L2 flush
 outside its CUDA-event interval: a 512 MB write, then a read of 256 MB of
 it, so that the step starts with none of the previous step's lines in L2
 and no dirty line either (write-backs of the flush would otherwise take
-about 20 us of HBM time from the first kernel of the step); barrier + synchronize
+about 20 us of HBM time from the first kernel of the step); then a 0.5 ms
+spin kernel, during which the host queues the step, so that the interval
+times the step's kernels and not the host's launch latency (a decode step
+is a quarter of a millisecond; serving replays it from a CUDA graph); barrier + synchronize
 around the timed region; the max over ranks.  Multi-GPU runs are weak
 scaling: every rank processes its own copy of the workload (independent
 sequences), no collective on the data path.
@@ -93,6 +96,9 @@ def algorithmic_work(wl):
         "attn_flop": c.H * (2.0 * c.D_K + 2.0 * c.D_V) * sel,
         "attn_bytes": 2.0 * c.D_K * sel,
     }
+
+
+SPIN_CYCLES = 1_000_000  # about 0.5 ms at 1.9-2 GHz, longer than the host takes to queue a step
 
 
 def slab_rows(wl):
@@ -205,6 +211,10 @@ def run_device(cid, steps, warmup, rank, world, do_e2e=True):
     for i in range(steps):
         flush.fill_(float(i))
         flush[: 64 << 20].sum()  # 256 MB read: the write-backs happen here
+        # a spin kernel keeps the GPU busy while the host queues the step, so
+        # the timed interval holds the step's kernels and not host launch
+        # latency (the e2e figure, which calls the API per step, includes it)
+        torch.cuda._sleep(SPIN_CYCLES)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         kinds, nl = step(evs)
@@ -516,6 +526,7 @@ def main():
             "data": "synthetic",
             "config": {"workload": DESCR[cid], "tokens_per_step_per_gpu": tokens,
                        "k": cfg.k, "l2": "flushed before every timed step (512 MB write, 256 MB of it read back)",
+                       "queued": "step launches queued behind a 0.5 ms spin kernel outside the timed interval",
                        "parallelism": f"{world} independent replicas (weak scaling)"},
             "roofline": roof, "stage_share": shares,
             "gpu_launches": launches,
