@@ -133,19 +133,6 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t sbo) {
   return d;
 }
 
-// K-major operand in the 64-byte-swizzled layout: rows of 64 bytes, 8-row
-// groups of 512 bytes, groups `sbo` bytes apart along M/N.  The tile base
-// must be 512-aligned; advancing K inside a row adds the byte offset.
-__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
-  d |= (uint64_t)1 << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)4 << 61;                   // 64-byte swizzle
-  return d;
-}
-
 // Same layout as desc_sw128, MN-major (the contiguous 128-byte rows run along M/N):
 // `lbo` = bytes between 64-element (128 B) column blocks along M/N,
 // `sbo` = bytes between 8-row groups along K.
