@@ -78,6 +78,16 @@ def test_argument_validation_without_device(lib):
     assert f(ctypes.byref(L), P, P, P, 4, 129, 576, 512, 0.1, P, None, None, 0, None) == E
     assert f(ctypes.byref(L), P, P, P, 4, 128, 576, 580, 0.1, P, None, None, 0, None) == E
     assert f(ctypes.byref(L), P, P, P, 4, 8, 80, 64, float("nan"), P, None, None, 0, None) == E
+    # chunked prefill: query offsets required, and no more queries than cache rows
+    ch = _layout(mode=dsa.DSA_CHUNKED, n_q=4)
+    assert lib.dsa_topk(ctypes.byref(ch), P, 4, P, None) == E  # q_offsets missing
+    ch_bad = _layout(mode=dsa.DSA_CHUNKED, n_q=9)
+    ch_bad.q_offsets = P
+    assert lib.dsa_topk(ctypes.byref(ch_bad), P, 4, P, None) == E  # n_q > n_k
+    ch_bad.q_offsets = P + 4
+    assert lib.dsa_indexer_scores(ctypes.byref(ch_bad), P, None, P, P, None, dsa.DSA_BF16, 64,
+                                  128, P, None) == E  # misaligned offsets
+    assert lib.dsa_topk(ctypes.byref(_layout(mode=3)), P, 4, P, None) == E  # unknown mode
     # the wait-timeout self-test takes limits in 0 .. 2e9 cycles only
     assert lib.dsa_selftest_wait_timeout(-1, None) == E
     assert lib.dsa_selftest_wait_timeout(2_000_000_001, None) == E
