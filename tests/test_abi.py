@@ -84,8 +84,9 @@ def test_argument_validation_without_device(lib):
     ch_bad = _layout(mode=dsa.DSA_CHUNKED, n_q=9)
     ch_bad.q_offsets = P
     assert lib.dsa_topk(ctypes.byref(ch_bad), P, 4, P, None) == E  # n_q > n_k
-    ch_bad.q_offsets = P + 4
-    assert lib.dsa_indexer_scores(ctypes.byref(ch_bad), P, None, P, P, None, dsa.DSA_BF16, 64,
+    ch_mis = _layout(mode=dsa.DSA_CHUNKED, n_q=4)
+    ch_mis.q_offsets = P + 4
+    assert lib.dsa_indexer_scores(ctypes.byref(ch_mis), P, None, P, P, None, dsa.DSA_BF16, 64,
                                   128, P, None) == E  # misaligned offsets
     assert lib.dsa_topk(ctypes.byref(_layout(mode=3)), P, 4, P, None) == E  # unknown mode
     # the wait-timeout self-test takes limits in 0 .. 2e9 cycles only
