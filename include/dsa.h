@@ -226,6 +226,45 @@ dsa_status_t dsa_forward_timed(const dsa_layout_t* layout, const dsa_forward_arg
                                int32_t n_events, int32_t* kinds, int32_t* n_launched);
 
 /*
+ * dsa_forward for inputs and results in host memory, pipelined over slabs of
+ * query rows: slab i's query rows are copied up (on a copy stream of the
+ * library's own) while slab i-1 computes on `stream` and slab i-2's output
+ * is copied down (on a second copy stream), so the two PCIe directions and
+ * the kernels overlap.  The kernels and their arguments are those of
+ * dsa_forward, and so are the results, up to the rounding order of the
+ * attention sums (the order of a row's selected indices is unspecified, as
+ * for dsa_topk, so two calls of either entry point may differ in the last
+ * bits).
+ *  host: the arguments with host pointers (pinned memory for the copies to
+ *        overlap; pageable memory gives the same results, serialised).
+ *        q_idx, w, q (and q_scale for e4m3) are required when n_q > 0.
+ *        k_idx, k_scale, kv may each be NULL: `dev`'s copy is then taken as
+ *        current (a cache kept in HBM across calls); otherwise all n_k rows
+ *        are copied before the first slab.  Scalars must equal dev's.
+ *  dev:  the same arguments with full-size device buffers (checked as in
+ *        dsa_forward); the call writes the host inputs into them.
+ *  host_out [n_q, H, D_V] bf16, host_lse [n_q, H] fp32 or NULL: the results;
+ *  dev_out / dev_lse: full-size device buffers they pass through (dev_lse
+ *        required when host_lse is given).
+ *  rows_per_slab: 0 for dsa_forward's slabs (bounded by 1 GiB of scores),
+ *        else at most that many rows per slab.
+ *  workspace: dsa_forward_host_workspace_size(layout, dev, rows_per_slab)
+ *        bytes, 16-byte aligned.
+ * Ordering: the copies start after the work `stream` holds at the call, and
+ * `stream` continues only after the last result reached host memory, so a
+ * synchronisation of `stream` makes host_out / host_lse readable.  With
+ * n_q = 0 nothing is copied or launched.  Errors: those of dsa_forward, and
+ * DSA_ERR_INVALID_ARGUMENT for host arguments that break the above.  After
+ * DSA_ERR_CUDA, copies may still be in flight: synchronise the device.
+ */
+size_t dsa_forward_host_workspace_size(const dsa_layout_t* layout, const dsa_forward_args_t* args,
+                                       int32_t rows_per_slab);
+dsa_status_t dsa_forward_host(const dsa_layout_t* layout, const dsa_forward_args_t* host,
+                              const dsa_forward_args_t* dev, void* host_out, float* host_lse,
+                              void* dev_out, float* dev_lse, int32_t rows_per_slab,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears this device's status word:
  * DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_DATA (DSA_ERR_CUDA if the
  * synchronisation itself failed).  The word is shared by every stream of the

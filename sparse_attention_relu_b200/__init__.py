@@ -77,6 +77,9 @@ def lib():
         L.dsa_forward_workspace_size.restype = SZ
         L.dsa_forward.argtypes = [LP, AP, P, P, P, P, SZ, P]
         L.dsa_forward_timed.argtypes = [LP, AP, P, P, P, P, SZ, P, P, I32, P, P]
+        L.dsa_forward_host_workspace_size.argtypes = [LP, AP, I32]
+        L.dsa_forward_host_workspace_size.restype = SZ
+        L.dsa_forward_host.argtypes = [LP, AP, AP, P, P, P, P, I32, P, SZ, P]
         L.dsa_device_status.argtypes = [P]
         L.dsa_selftest_wait_timeout.argtypes = [I64, P]
         L.dsa_status_string.argtypes = [ctypes.c_int]
@@ -84,7 +87,8 @@ def lib():
         L.dsa_abi_version.restype = I32
         for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn",
                      "dsa_sparse_mla_attn_noalloc", "dsa_forward",
-                     "dsa_forward_timed", "dsa_device_status", "dsa_selftest_wait_timeout"):
+                     "dsa_forward_timed", "dsa_forward_host", "dsa_device_status",
+                     "dsa_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -189,12 +193,25 @@ def dsa_sparse_mla_attn_noalloc(layout: Layout, q, kv, idx, k: int, D_V: int, sm
     return out
 
 
-def forward_args(*, q_idx, q_scale, w, k_idx, k_scale, q, kv, D_V, sm_scale, k):
+def _hptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("expected a host tensor")
+    if not t.is_contiguous():
+        raise ValueError("libdsa takes contiguous tensors")
+    return t.data_ptr() or None
+
+
+def forward_args(*, q_idx, q_scale, w, k_idx, k_scale, q, kv, D_V, sm_scale, k, host=False):
+    """The argument block of dsa_forward; host=True takes host tensors (the
+    `host` block of dsa_forward_host, where k_idx / k_scale / kv may be None)."""
     n_q, H_I, D_I = q_idx.shape
     _, H, D_K = q.shape
-    a = dsa_forward_args_t(_DTYPE_CODE[q_idx.dtype], H_I, D_I, _ptr(q_idx), _ptr(q_scale), _ptr(w),
-                           _ptr(k_idx), _ptr(k_scale), H, D_K, int(D_V), float(sm_scale), _ptr(q),
-                           _ptr(kv), int(k))
+    f = _hptr if host else _ptr
+    a = dsa_forward_args_t(_DTYPE_CODE[q_idx.dtype], H_I, D_I, f(q_idx), f(q_scale), f(w),
+                           f(k_idx), f(k_scale), H, D_K, int(D_V), float(sm_scale), f(q),
+                           f(kv), int(k))
     a._keep = (q_idx, q_scale, w, k_idx, k_scale, q, kv)
     return a
 
@@ -232,6 +249,24 @@ def dsa_forward_timed(layout: Layout, args: dsa_forward_args_t, out, lse, idx_ou
                                    _ptr(idx_out), _ptr(workspace), ws_bytes, _stream(stream), arr,
                                    n, kinds, ctypes.byref(nl)), "dsa_forward_timed")
     return [kinds[i] for i in range(min(nl.value, max(n - 1, 0)))], nl.value
+
+
+def dsa_forward_host_workspace_size(layout: Layout, args: dsa_forward_args_t,
+                                    rows_per_slab: int = 0) -> int:
+    return lib().dsa_forward_host_workspace_size(layout.ref, ctypes.byref(args),
+                                                 int(rows_per_slab))
+
+
+def dsa_forward_host(layout: Layout, host: dsa_forward_args_t, dev: dsa_forward_args_t, host_out,
+                     host_lse, dev_out, dev_lse, workspace, rows_per_slab: int = 0, stream=None):
+    """The whole chain from host inputs to host results, copies and kernels
+    overlapped slab by slab; `stream` is done once host_out is written."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().dsa_forward_host(layout.ref, ctypes.byref(host), ctypes.byref(dev),
+                                  _hptr(host_out), _hptr(host_lse), _ptr(dev_out), _ptr(dev_lse),
+                                  int(rows_per_slab), _ptr(workspace), ws_bytes, _stream(stream)),
+           "dsa_forward_host")
+    return host_out
 
 
 def dsa_selftest_wait_timeout(cycles: int, stream=None):

@@ -154,9 +154,12 @@ struct ForwardPlan {
   size_t off_scores, off_idx, off_attn, total;
 };
 
-ForwardPlan plan_forward(const Rows& R, const dsa_forward_args_t* a, bool own_idx) {
+// slab_cap > 0 caps the rows per slab below the scores bound.
+ForwardPlan plan_forward(const Rows& R, const dsa_forward_args_t* a, bool own_idx,
+                         int32_t slab_cap = 0) {
   ForwardPlan p{};
   p.slab = slab_rows(R);
+  if (slab_cap > 0 && slab_cap < p.slab) p.slab = slab_cap;
   size_t o = 0;
   p.off_scores = o;
   o = align_up(o + (size_t)p.slab * R.max_len * 4);
@@ -168,6 +171,53 @@ ForwardPlan plan_forward(const Rows& R, const dsa_forward_args_t* a, bool own_id
   return p;
 }
 
+// The two copy streams of dsa_forward_host (host to device, device to host),
+// one pair per device, created on first use and kept for the process.
+dsa_status_t copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
+  static cudaStream_t made[64][2] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DSA_ERR_CUDA;
+  for (int i = 0; i < 2; ++i)
+    if (!made[dev][i] &&
+        cudaStreamCreateWithFlags(&made[dev][i], cudaStreamNonBlocking) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  *h2d = made[dev][0];
+  *d2h = made[dev][1];
+  return DSA_OK;
+}
+
+// Host-side arguments of dsa_forward_host: the same shapes and scalars as the
+// device ones; every per-query input present (q_scale exactly when e4m3); a
+// key-side input may be NULL (its device copy is current).
+dsa_status_t check_host(const Rows& R, const dsa_forward_args_t* h, const dsa_forward_args_t* d,
+                        const void* host_out, const float* host_lse, const float* dev_lse) {
+  if (h->idx_dtype != d->idx_dtype || h->H_I != d->H_I || h->D_I != d->D_I || h->H != d->H ||
+      h->D_K != d->D_K || h->D_V != d->D_V || h->k != d->k || !(h->sm_scale == d->sm_scale))
+    return DSA_ERR_INVALID_ARGUMENT;
+  const bool rows = R.n_q > 0, e4m3 = d->idx_dtype == DSA_E4M3;
+  if (rows && (!h->q_idx || !h->w || !h->q || !host_out || (e4m3 && !h->q_scale)))
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!e4m3 && (h->q_scale || h->k_scale)) return DSA_ERR_INVALID_ARGUMENT;
+  if (host_lse && !dev_lse) return DSA_ERR_INVALID_ARGUMENT;
+  return DSA_OK;
+}
+
+// Events of one dsa_forward_host call, destroyed on return (a recorded event
+// that has not completed is released by the runtime once it completes; waits
+// already enqueued on it are unaffected).
+struct CallEvents {
+  cudaEvent_t e[4] = {};
+  bool ok = true;
+  CallEvents() {
+    for (auto& x : e)
+      if (cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess) ok = false;
+  }
+  ~CallEvents() {
+    for (auto& x : e)
+      if (x) cudaEventDestroy(x);
+  }
+};
+
 }  // namespace
 }  // namespace dsa
 
@@ -175,7 +225,7 @@ using namespace dsa;
 
 extern "C" {
 
-int32_t dsa_abi_version(void) { return 2; }
+int32_t dsa_abi_version(void) { return 3; }
 
 const char* dsa_status_string(dsa_status_t s) {
   switch (s) {
@@ -349,6 +399,91 @@ dsa_status_t dsa_forward(const dsa_layout_t* layout, const dsa_forward_args_t* a
                          void* stream) {
   return dsa_forward_timed(layout, a, out, lse, idx_out, workspace, ws_bytes, stream, nullptr, 0,
                            nullptr, nullptr);
+}
+
+size_t dsa_forward_host_workspace_size(const dsa_layout_t* layout, const dsa_forward_args_t* a,
+                                       int32_t rows_per_slab) {
+  Rows R;
+  if (!a || rows_per_slab < 0 || check_layout(layout, &R)) return 0;
+  return plan_forward(R, a, true, rows_per_slab).total;
+}
+
+dsa_status_t dsa_forward_host(const dsa_layout_t* layout, const dsa_forward_args_t* host,
+                              const dsa_forward_args_t* dev, void* host_out, float* host_lse,
+                              void* dev_out, float* dev_lse, int32_t rows_per_slab,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  Rows R;
+  dsa_status_t s = check_layout(layout, &R);
+  if (s) return s;
+  if (!host || !dev || rows_per_slab < 0) return DSA_ERR_INVALID_ARGUMENT;
+  const dsa_forward_args_t* a = dev;
+  if ((s = check_indexer(R, a->q_idx, a->q_scale, a->w, a->k_idx, a->k_scale, a->idx_dtype,
+                         a->H_I, a->D_I)))
+    return s;
+  if ((s = check_attn(R, a->q, a->kv, a->k, a->H, a->D_K, a->D_V, a->sm_scale, dev_out,
+                      dev_lse)))
+    return s;
+  if ((s = check_host(R, host, dev, host_out, host_lse, dev_lse))) return s;
+  const ForwardPlan p = plan_forward(R, a, true, rows_per_slab);
+  if (!workspace || ws_bytes < p.total || !aligned16(workspace)) return DSA_ERR_WORKSPACE;
+  if (R.n_q == 0) return DSA_OK;
+  if ((s = device_rows(&R))) return s;
+  cudaStream_t st = (cudaStream_t)stream, hs = nullptr, ds = nullptr;
+  if ((s = copy_streams(&hs, &ds))) return s;
+  CallEvents ev;
+  if (!ev.ok) return DSA_ERR_CUDA;
+  const cudaEvent_t start = ev.e[0], in = ev.e[1], done = ev.e[2], end = ev.e[3];
+  // bytes of one row of each array
+  const size_t esz = a->idx_dtype == DSA_F32 ? 4 : a->idx_dtype == DSA_BF16 ? 2 : 1;
+  const size_t qi_row = (size_t)a->H_I * a->D_I * esz, hv_row = (size_t)a->H_I * 4,
+               q_row = (size_t)a->H * a->D_K * 2, out_row = (size_t)a->H * a->D_V * 2,
+               lse_row = (size_t)a->H * 4;
+  // bytes [off, off + n) of src to dst on cs; nothing when either side is absent
+  auto copy = [](const void* dst, const void* src, size_t off, size_t n, cudaStream_t cs) {
+    return !dst || !src || !n ||
+           cudaMemcpyAsync((char*)dst + off, (const char*)src + off, n, cudaMemcpyDefault, cs) ==
+               cudaSuccess;
+  };
+  char* ws = (char*)workspace;
+  float* scores = (float*)(ws + p.off_scores);
+  int32_t* idx = (int32_t*)(ws + p.off_idx);
+  // the copies start after what `stream` holds (the previous call included)
+  bool ok = cudaEventRecord(start, st) == cudaSuccess &&
+            cudaStreamWaitEvent(hs, start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(ds, start, 0) == cudaSuccess;
+  // the key side first: any slab may read any cache row
+  ok = ok && copy(a->k_idx, host->k_idx, 0, (size_t)R.n_k * a->D_I * esz, hs) &&
+       copy(a->k_scale, host->k_scale, 0, (size_t)R.n_k * 4, hs) &&
+       copy(a->kv, host->kv, 0, (size_t)R.n_k * a->D_K * 2, hs);
+  for (int32_t r0 = 0; ok && r0 < R.n_q; r0 += p.slab) {
+    const int32_t nr = (R.n_q - r0) < p.slab ? (R.n_q - r0) : p.slab;
+    const size_t r = (size_t)r0, n = (size_t)nr;
+    // slab i's query rows go up while slab i-1 computes and slab i-2's results come down
+    ok = copy(a->q_idx, host->q_idx, r * qi_row, n * qi_row, hs) &&
+         copy(a->q_scale, host->q_scale, r * hv_row, n * hv_row, hs) &&
+         copy(a->w, host->w, r * hv_row, n * hv_row, hs) &&
+         copy(a->q, host->q, r * q_row, n * q_row, hs) && cudaEventRecord(in, hs) == cudaSuccess &&
+         cudaStreamWaitEvent(st, in, 0) == cudaSuccess;
+    if (!ok) break;
+    if ((s = run_indexer(R, r0, nr, a->idx_dtype, a->H_I, a->D_I, a->q_idx, a->q_scale, a->w,
+                         a->k_idx, a->k_scale, scores, false, st)))
+      break;
+    if ((s = launch_topk(R, r0, nr, scores, R.max_len, a->k, idx, st))) break;
+    if ((s = run_attn(R, r0, nr, a->q, a->kv, idx, a->k, a->H, a->D_K, a->D_V, a->sm_scale,
+                      dev_out, dev_lse, ws + p.off_attn, p.total - p.off_attn, st)))
+      break;
+    ok = cudaEventRecord(done, st) == cudaSuccess &&
+         cudaStreamWaitEvent(ds, done, 0) == cudaSuccess &&
+         copy(host_out, dev_out, r * out_row, n * out_row, ds) &&
+         copy(host_lse, dev_lse, r * lse_row, n * lse_row, ds);
+  }
+  // join, on every path: `stream` goes on only after both copy streams drained
+  const bool joined = cudaEventRecord(in, hs) == cudaSuccess &&
+                      cudaStreamWaitEvent(st, in, 0) == cudaSuccess &&
+                      cudaEventRecord(end, ds) == cudaSuccess &&
+                      cudaStreamWaitEvent(st, end, 0) == cudaSuccess;
+  if (s) return s;
+  return ok && joined ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -95,3 +95,37 @@ def test_argument_validation_without_device(lib):
     # empty problems succeed without launching anything
     empty = _layout(batch=0, kv_offsets=None, max_len=0, n_q=0, n_k=0)
     assert lib.dsa_topk(ctypes.byref(empty), None, 4, None, None) == dsa.DSA_OK
+
+
+def test_forward_host_validation_without_device(lib):
+    """dsa_forward_host checks its host block against the device block before
+    any copy or launch."""
+    E = dsa.DSA_ERR_INVALID_ARGUMENT
+    P, H = 4096, 8192  # fake device / host addresses: never dereferenced
+    L = _layout()
+
+    def args(ptr, **kw):
+        d = dict(idx_dtype=dsa.DSA_BF16, H_I=64, D_I=128, q_idx=ptr, q_scale=None, w=ptr,
+                 k_idx=ptr, k_scale=None, H=128, D_K=576, D_V=512, sm_scale=0.1, q=ptr, kv=ptr,
+                 k=4)
+        d.update(kw)
+        return dsa.dsa_forward_args_t(*d.values())
+
+    dev = args(P)
+
+    def call(host, rows=0, host_lse=None, dev_lse=None, dev_args=dev):
+        return lib.dsa_forward_host(ctypes.byref(L), None if host is None else ctypes.byref(host),
+                                    ctypes.byref(dev_args), H, host_lse, P, dev_lse, rows, P,
+                                    1 << 30, None)
+
+    assert call(None) == E
+    assert call(args(H), rows=-1) == E
+    assert call(args(H, H_I=32)) == E  # scalars differ from the device block
+    assert call(args(H, sm_scale=0.2)) == E
+    assert call(args(H, q=None)) == E  # a per-query input missing
+    assert call(args(H, w=None)) == E
+    assert call(args(H, k_scale=H)) == E  # scales only with e4m3
+    assert call(args(H), host_lse=H) == E  # host lse without a device lse
+    e4 = args(P, idx_dtype=dsa.DSA_E4M3, q_scale=P, k_scale=P)
+    assert call(args(H, idx_dtype=dsa.DSA_E4M3, k_scale=H), dev_args=e4) == E  # q_scale missing
+    assert lib.dsa_forward_host_workspace_size(ctypes.byref(L), ctypes.byref(dev), -1) == 0
