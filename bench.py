@@ -283,28 +283,32 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
                             kv=dbuf["kv"], D_V=c.D_V, sm_scale=c.sm_scale, k=c.k)
     out = torch.empty(wl.n_q, c.H, c.D_V, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(wl.n_q, c.H, dtype=torch.float32, device=dev)
-    if not resident:
-        # every input comes from the host: dsa_forward_host overlaps the
-        # uploads, the kernels and the downloads slab by slab
+    # prefill and chunked prefill run several slabs: dsa_forward_host overlaps
+    # the query uploads, the kernels and the output downloads slab by slab (a
+    # resident cache is passed as NULL on the host side); decode is one slab
+    use_host = c.mode != "decode"
+    if use_host:
         hargs = dsa.forward_args(q_idx=host["q_idx"], q_scale=host.get("q_scale"), w=host["w"],
-                                 k_idx=host["k_idx"], k_scale=host.get("k_scale"), q=host["q"],
-                                 kv=host["kv"], D_V=c.D_V, sm_scale=c.sm_scale, k=c.k, host=True)
+                                 k_idx=host.get("k_idx"), k_scale=host.get("k_scale"),
+                                 q=host["q"], kv=host.get("kv"), D_V=c.D_V, sm_scale=c.sm_scale,
+                                 k=c.k, host=True)
         nws = dsa.dsa_forward_host_workspace_size(lay2, args)
         if nws > ws.numel():
             ws = torch.empty(nws, dtype=torch.uint8, device=dev)
 
     def one():
-        if not resident:
-            dsa.dsa_forward_host(lay2, hargs, args, out_h, lse_h, out, lse, ws)
-            return
-        for n, t in host.items():
-            dbuf[n].copy_(t, non_blocking=True)
+        if not use_host:
+            for n, t in host.items():
+                dbuf[n].copy_(t, non_blocking=True)
         for n, (h, stage) in new_rows.items():  # the new tokens' cache rows, in place
             stage.copy_(h, non_blocking=True)
             if stage.dtype == torch.float8_e4m3fn:  # no fp8 index_copy: move the bytes
                 dbuf[n].view(torch.uint8).index_copy_(0, last_dev, stage.view(torch.uint8))
             else:
                 dbuf[n].index_copy_(0, last_dev, stage)
+        if use_host:
+            dsa.dsa_forward_host(lay2, hargs, args, out_h, lse_h, out, lse, ws)
+            return
         dsa.dsa_forward(lay2, args, out, lse, None, ws)
         out_h.copy_(out, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
@@ -319,8 +323,9 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
     e1.synchronize()
     ms = e0.elapsed_time(e1) / steps
     inputs = ("new queries + the new tokens' cache rows per step (caches resident in HBM)"
-              if cache else "every input of the step (queries, indexer keys, MLA cache), "
-              "copies overlapped with the kernels slab by slab (dsa_forward_host)")
+              if cache else "every input of the step (queries, indexer keys, MLA cache)")
+    if use_host:
+        inputs += "; copies overlapped with the kernels slab by slab (dsa_forward_host)"
     return {"ms_per_step": ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "inputs": inputs}
 
