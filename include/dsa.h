@@ -253,7 +253,9 @@ dsa_status_t dsa_forward_timed(const dsa_layout_t* layout, const dsa_forward_arg
  * Ordering: the copies start after the work `stream` holds at the call, and
  * `stream` continues only after the last result reached host memory, so a
  * synchronisation of `stream` makes host_out / host_lse readable.  With
- * n_q = 0 nothing is copied or launched.  Errors: those of dsa_forward, and
+ * n_q = 0 nothing is copied or launched.  Calls from several host threads
+ * are correct; their copies share the device's two copy streams, so they
+ * take turns on PCIe.  Errors: those of dsa_forward, and
  * DSA_ERR_INVALID_ARGUMENT for host arguments that break the above.  After
  * DSA_ERR_CUDA, copies may still be in flight: synchronise the device.
  */

@@ -2,6 +2,8 @@
 // The semantics of each call are documented in include/dsa.h.
 #include <math.h>
 
+#include <mutex>
+
 #include "kernels.cuh"
 #include "sm100.cuh"
 
@@ -172,9 +174,12 @@ ForwardPlan plan_forward(const Rows& R, const dsa_forward_args_t* a, bool own_id
 }
 
 // The two copy streams of dsa_forward_host (host to device, device to host),
-// one pair per device, created on first use and kept for the process.
+// one pair per device, created on first use and kept for the process.  The
+// lock makes the first use from several host threads create one pair.
 dsa_status_t copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
   static cudaStream_t made[64][2] = {};
+  static std::mutex lock;
+  std::lock_guard<std::mutex> hold(lock);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DSA_ERR_CUDA;
   for (int i = 0; i < 2; ++i)
