@@ -10,8 +10,11 @@
  *
  * Conventions shared by every call
  *  - Tensor arguments are DEVICE pointers owned by the caller; the library
- *    never allocates, frees or synchronises (dsa_device_status excepted).
- *    Scratch memory comes only through the caller's `workspace`.
+ *    never allocates device memory, frees or synchronises (dsa_device_status
+ *    excepted).  Scratch memory comes only through the caller's `workspace`.
+ *    dsa_forward_host alone also takes HOST pointers (its `host` block and
+ *    results), and creates two copy streams per device on first use and a
+ *    few events per call.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
  *    only enqueues work on it and returns.
  *  - Arguments are validated on the host before anything is launched; a
@@ -22,7 +25,8 @@
  *    exceed n_k, an index outside its sequence, a bounded wait that ran out)
  *    make the kernels skip the affected row or tile and raise a bit in a
  *    per-device status word, read and cleared by dsa_device_status().
- *  - Every pointer passed must be 16-byte aligned.
+ *  - Every device pointer passed must be 16-byte aligned (host pointers may
+ *    have any alignment).
  *  - Index outputs are LOCAL positions inside the query's own sequence.
  *  - bf16 tensors are passed as raw 16-bit storage, e4m3 as raw bytes
  *    (OCP FP8 E4M3 "fn": no infinities, S.1111.111 = NaN).
@@ -125,8 +129,9 @@ dsa_status_t dsa_topk(const dsa_layout_t* layout, const float* scores, int32_t k
 /*
  * Stage 3, sparse MLA attention ("GLM sparse attention", MLA passage: one
  * latent row per token, read by every head as in multi-query attention, and
- * "exact softmax over the survivors"; "DeepSeek Sparse Attention"
- * (divagr.pages.dev), "the risk": an excluded token contributes nothing):
+ * a full softmax over the selected tokens, the attention itself not
+ * approximated; "DeepSeek Sparse Attention" (divagr.pages.dev), "the risk":
+ * a token left out of the selection adds nothing to the output):
  *
  *   z[h, s]  = sm_scale * <q[r, h, 0:D_K], kv[kbase + s, 0:D_K]>
  *   out[r,h] = sum_{s in S_r} softmax_S(z[h, :])_s * kv[kbase + s, 0:D_V]

@@ -29,7 +29,7 @@
  *    "Top-K Selection": k = 2048.
  *  - "DeepSeek Sparse Attention" (divagr.pages.dev), "The lightning
  *    indexer": scores rank positions and are not attention weights; "the
- *    risk": an excluded token cannot contribute.
+ *    risk": a token left out of the selection adds nothing to the output.
  *
  * Readings where the pages are silent (each repeated beside its code):
  *  - candidates of query t are the positions s <= t of its own sequence;

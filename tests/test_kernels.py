@@ -142,8 +142,8 @@ def test_attention_edge_cases():
 
 def test_unselected_rows_do_not_contribute():
     """Poisoning every unselected cache row with NaN leaves the output
-    bit-identical ("DeepSeek Sparse Attention", the risk: an excluded token
-    cannot contribute)."""
+    bit-identical ("DeepSeek Sparse Attention", section on the risk: a token
+    left out of the selection adds nothing to the output)."""
     cfg = workloads.custom("prefill", [400], idx_dtype="bf16", k=64)
     dev = Dev(workloads.generate(cfg))
     idx = dev.topk(dev.scores())
