@@ -23,8 +23,8 @@
  *    clips each negative similarity to zero before the weighted sum; the
  *    threshold figure: the cut-off is the k-th best score; MLA passage: one
  *    cached latent plus one decoupled rotary key per token, scored directly by
- *    absorbed queries, shared by every head; "exact softmax over the
- *    survivors".
+ *    absorbed queries, shared by every head; a full softmax over the
+ *    selected tokens, with nothing approximated in the attention itself.
  *  - "Sparse Attention Architecture Evolution in LLMs" (intl.cloud.baidu.com),
  *    "Top-K Selection": k = 2048.
  *  - "DeepSeek Sparse Attention" (divagr.pages.dev), "The lightning

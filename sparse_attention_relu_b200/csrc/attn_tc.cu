@@ -5,8 +5,8 @@
 //   o[r,h] = sum_s softmax_S(z[h,:])_s * C[s,0:512],   lse = log sum_s exp z
 // ("GLM sparse attention", MLA passage: one cached latent row (512 latent +
 // 64 rotary) per token, scored by the absorbed query of every head, so one
-// gathered row serves all 128 heads; exact softmax over the survivors; the
-// selected positions are scattered, so the gather must be efficient.)
+// gathered row serves all 128 heads; a full softmax over the selected rows;
+// these rows lie anywhere in the cache, so the gather sets the pace.)
 //
 // TMEM holds 128 lanes x 512 fp32 columns, exactly the size of the 128 x 512
 // output accumulator.  Each query row therefore runs on two CTAs, one per
