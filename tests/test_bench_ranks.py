@@ -61,3 +61,30 @@ def test_single_rank_is_identity():
 
     assert bench.max_over_ranks(3.25, 1, "cpu") == 3.25
     assert bench.job_throughput(100, 10.0, 1) == pytest.approx(10000.0)
+
+
+def _bench(args, env_extra):
+    import json
+    import subprocess
+
+    env = dict(os.environ, **env_extra)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    return [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_reference_arm_line_on_the_host():
+    """--impl reference times the oracle on the host cores (no GPU needed) and
+    prints one line with the arm's own metric, cpu_baseline and e2e."""
+    args = ["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "3"]
+    (line,) = _bench(args, {"RANK": "0", "WORLD_SIZE": "1"})
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s"
+    assert line["higher_is_better"] is True and line["value"] > 0
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+    # under torchrun only rank 0 runs it: another rank prints nothing and exits 0
+    assert _bench(args, {"RANK": "1", "WORLD_SIZE": "2"}) == []
