@@ -207,9 +207,10 @@ typedef struct {
 size_t dsa_forward_workspace_size(const dsa_layout_t* layout, const dsa_forward_args_t* args);
 
 /*
- * The whole hot path, prefill or decode: indexer -> top-k -> sparse MLA
- * attention, enqueued on one stream.  Prefill processes query rows in slabs
- * so that only a slab of scores is ever held (in the workspace).
+ * The whole hot path (prefill, chunked or decode): indexer -> top-k -> sparse MLA
+ * attention, enqueued on one stream.  Query rows run in slabs so that only a
+ * slab of scores is ever held (in the workspace): as many rows as fit 1 GiB
+ * of fp32 scores at max_len per row (4096 rows at 64K context).
  *  out [n_q, H, D_V] bf16; lse [n_q, H] fp32 or NULL;
  *  idx_out [n_q, k] int32 or NULL (then the indices live in the workspace).
  */
