@@ -129,3 +129,25 @@ def test_forward_host_validation_without_device(lib):
     e4 = args(P, idx_dtype=dsa.DSA_E4M3, q_scale=P, k_scale=P)
     assert call(args(H, idx_dtype=dsa.DSA_E4M3, k_scale=H), dev_args=e4) == E  # q_scale missing
     assert lib.dsa_forward_host_workspace_size(ctypes.byref(L), ctypes.byref(dev), -1) == 0
+
+
+def test_binding_fails_loudly_without_device_or_library(monkeypatch, lib):
+    """No CPU fallback: host tensors are refused where the ABI takes device
+    pointers, and a missing library is an error, not a silent substitute."""
+    import torch
+
+    offs = torch.tensor([0, 8], dtype=torch.int32)  # a host tensor
+    with pytest.raises(ValueError, match="device tensors"):
+        dsa.Layout(offs, dsa.DSA_PREFILL, 8, 8, 8)
+    with pytest.raises(ValueError, match="device tensors"):
+        dsa.forward_args(q_idx=torch.zeros(8, 4, 32), q_scale=None, w=torch.zeros(8, 4),
+                         k_idx=torch.zeros(8, 32), k_scale=None, q=torch.zeros(8, 8, 80),
+                         kv=torch.zeros(8, 80), D_V=64, sm_scale=0.1, k=4)
+    with pytest.raises(ValueError, match="contiguous"):  # the host block of dsa_forward_host
+        dsa.forward_args(q_idx=torch.zeros(8, 32, 4).transpose(1, 2), q_scale=None,
+                         w=torch.zeros(8, 4), k_idx=None, k_scale=None, q=torch.zeros(8, 8, 80),
+                         kv=None, D_V=64, sm_scale=0.1, k=4, host=True)
+    monkeypatch.setattr(dsa, "_lib", None)
+    monkeypatch.setattr(dsa, "LIB_PATH", os.path.join(ROOT, "no_such_libdsa.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        dsa.lib()
