@@ -224,6 +224,49 @@ def test_topk_matches_stable_argsort(oracle_mod):
         assert np.array_equal(got[i], exp)
 
 
+def test_topk_f64_matches_stable_argsort(oracle_mod):
+    """The fp64 ranking (used on the oracle's own scores by every end-to-end
+    selection check) against numpy's stable argsort: ties to the lower
+    position ("Sparse Attention Architecture Evolution in LLMs", Top-K
+    Selection), rows shorter than the stride, values that differ below
+    float32 resolution, +0/-0 and NaN (ranked as -inf)."""
+    rng = np.random.default_rng(18)
+    n, ld, k = 40, 257, 31
+    s = np.round(rng.standard_normal((n, ld)) * 3).astype(np.float64)  # many ties
+    # differences float32 cannot see: the fp64 path must keep them apart
+    s[::3, ::5] += 1e-12 * rng.integers(1, 4, s[::3, ::5].shape)
+    s[1, :] = 0.0
+    s[1, 1::2] = -0.0  # +0 and -0 tie: position order
+    s[2, :] = -2.0
+    s[2, [3, 7, 100]] = np.nan  # NaN ranks as -inf: after every finite score
+    s[3, :] = -np.inf
+    s[3, [10, 20]] = np.nan  # NaN ties with -inf: position order
+    nv = rng.integers(1, ld + 1, n)
+    nv[1:4] = ld
+    nv[4] = 1
+    got = oracle_mod.topk(s, nv, k)
+    assert got.dtype == np.int32 and got.shape == (n, k)
+    for i in range(n):
+        key = np.where(np.isnan(s[i, : nv[i]]), -np.inf, s[i, : nv[i]])
+        order = np.argsort(-key, kind="stable")[:k]
+        exp = np.full(k, -1, np.int32)
+        exp[: len(order)] = order
+        assert np.array_equal(got[i], exp), f"row {i}"
+    assert list(got[1][:4]) == [0, 1, 2, 3]
+    assert not {3, 7, 100} & set(got[2].tolist())
+    assert list(got[3][:5]) == [0, 1, 2, 3, 4]
+    # a row read at the wrong stride would pick up the neighbour's values
+    t = np.full((3, 64), -5.0)
+    t[1, :16] = np.arange(16.0)
+    t[0, 16:] = 100.0  # past row 0's valid prefix: never read
+    got = oracle_mod.topk(t, np.array([16, 16, 16]), 4)
+    assert list(got[0]) == [0, 1, 2, 3] and list(got[1]) == [15, 14, 13, 12]
+    # fp64 resolution: a float32 cast would tie these and pick position order
+    u = np.array([[1.0, 1.0 + 1e-12, 1.0 + 2e-12, 1.0]])
+    assert list(oracle_mod.topk(u, np.array([4]), 2)[0]) == [2, 1]
+    assert list(oracle_mod.topk(u.astype(np.float32), np.array([4]), 2)[0]) == [0, 1]
+
+
 def test_topk_special_rows(oracle_mod):
     k = 8
     rows = np.zeros((5, 20), np.float32)
