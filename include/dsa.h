@@ -22,7 +22,7 @@
  *    DSA_ERR_WORKSPACE and leaves every output untouched.  A failed launch
  *    returns DSA_ERR_CUDA.
  *  - Conditions only the device can see (offsets that are not monotone or
- *    exceed n_k, an index outside its sequence, a bounded wait that ran out)
+ *    exceed n_k, an index outside its causal range, a bounded wait that ran out)
  *    make the kernels skip the affected row or tile and raise a bit in a
  *    per-device status word, read and cleared by dsa_device_status().
  *  - Every device pointer passed must be 16-byte aligned (host pointers may
@@ -138,7 +138,9 @@ dsa_status_t dsa_topk(const dsa_layout_t* layout, const float* scores, int32_t k
  *   lse[r,h] = log sum_{s in S_r} exp(z[h, s])          (natural log)
  *
  * S_r = the entries of idx[r, 0:k] that are >= 0 (-1 marks an empty slot);
- * entries must be distinct and < L_b.  q is the absorbed query (rope part
+ * entries must be distinct causal positions, 0 <= s <= t(r) (so < L_b); an
+ * entry outside that range is skipped like -1 and raises
+ * DSA_ERR_DEVICE_DATA.  q is the absorbed query (rope part
  * already rotated), kv a row of latent (first D_V columns, also the value)
  * followed by the rotary key.  A row with no selected position gets out = 0
  * and lse = -inf.

@@ -62,7 +62,8 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(Rows R, int32_t row
   for (int c0 = 0; c0 < k; c0 += kChunk) {
     if (tid < kChunk) {
       int s = (c0 + tid < k) ? __ldg(irow + c0 + tid) : -1;
-      if (s < -1 || s >= ri.len || ri.t < 0) {
+      // candidates are the causal positions 0..t (t < L_b); a later one is bad data
+      if (s < -1 || s > ri.t) {
         if (s != -1 && ri.t >= 0) raise_status(R, kErrBadIndex);
         s = -1;
       }

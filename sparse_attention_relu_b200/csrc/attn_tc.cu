@@ -318,7 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto load_idx = [&](int n) -> int32_t {
       const int slot = slot_lo + n * kNT + tid;
       int32_t s = slot < slot_hi ? __ldg(idx + (int64_t)rloc * k + slot) : -1;
-      if (s < -1 || s >= ri.len || ri.t < 0) {
+      // candidates are the causal positions 0..t (t < L_b); a later one is bad data
+      if (s < -1 || s > ri.t) {
         if (s != -1 && ri.t >= 0) raise_status(R, kErrBadIndex);
         s = -1;
       }
@@ -768,8 +769,10 @@ dsa_status_t launch_attn_tc_static(const Rows& R, int32_t row0, int32_t nrows, c
   void* scratch = nullptr;
   if (need) {
     static void* addr[64] = {};
+    static std::mutex lock;  // concurrent first calls from several host threads
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DSA_ERR_CUDA;
+    std::lock_guard<std::mutex> hold(lock);
     if (!addr[dev]) {
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;

@@ -14,10 +14,14 @@ namespace {
 // The per-device status word.  Kernels receive its device address in Rows.
 __device__ unsigned g_status = 0;
 
+// Its device address, looked up once per device with that device current;
+// the lock makes concurrent first calls from several host threads safe.
 unsigned* status_word() {
   static unsigned* addr[64] = {};
+  static std::mutex lock;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> hold(lock);
   if (!addr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;

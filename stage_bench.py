@@ -1,7 +1,7 @@
 """Times one stage of the hot path through its C ABI call on a synthetic case.
 
-    python -m sparse_attention_relu_b200.stage_bench --stage attn --case prefill --reps 4
-    python -m sparse_attention_relu_b200.stage_bench --stage indexer --case prefill --tokens 16384
+    python stage_bench.py --stage attn --case prefill --reps 4
+    python stage_bench.py --stage indexer --case prefill --tokens 16384
 
 Small, fixed cases meant for profiler captures of a single kernel:
   attn/prefill   one sequence of T tokens (cache L2-resident); row t selects
@@ -18,7 +18,7 @@ import sys
 
 import torch
 
-ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 

@@ -54,6 +54,31 @@ def test_index_outside_its_sequence_is_skipped_and_reported():
     assert_attn_close(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref)
 
 
+@pytest.mark.parametrize("shape", ["tensor_core", "generic"])
+def test_future_position_is_skipped_and_reported(shape):
+    """A prefill query may only attend to positions s <= t (the causal mask of
+    the indexer, "GLM sparse attention").  An index past t but inside the
+    sequence is dropped like -1 and raises DSA_ERR_DEVICE_DATA; both the
+    tensor-core kernel and the generic one check it."""
+    kw = {} if shape == "tensor_core" else dict(H_I=16, D_I=64, idx_dtype="f32", H=20, D_K=96,
+                                                D_V=32)
+    cfg = workloads.custom("prefill", [400], k=64, seed=9, **kw)
+    dev = Dev(workloads.generate(cfg))
+    idx = dev.topk(dev.scores())
+    assert dsa.dsa_device_status() == dsa.DSA_OK
+    bad = idx.clone()
+    bad[10, 0] = 11  # row 10 sees 0..10
+    bad[300, 5] = 399
+    out, lse = dev.attn(bad)
+    assert dsa.dsa_device_status() == dsa.DSA_ERR_DEVICE_DATA
+    ref_idx = bad.cpu().numpy().copy()
+    ref_idx[10, 0] = -1
+    ref_idx[300, 5] = -1
+    rows = np.arange(dev.wl.n_q)
+    o_ref, l_ref = ref_attn(dev.wl, rows, ref_idx)
+    assert_attn_close(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref)
+
+
 def test_offsets_past_the_cache_are_reported_and_the_rows_skipped():
     """A layout whose last offset runs past n_k: the indexer, top-k and
     attention skip that sequence (scores -inf, indices -1, output 0) and raise

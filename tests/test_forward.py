@@ -1,12 +1,17 @@
 """End-to-end parity of dsa_forward at the five workload sizes.
 
 Each workload runs in full on the GPU in the same launch configuration the
-benchmark times; the oracle checks a sample of query rows (evenly spaced,
-plus the first rows past k, the last row and the planted needles): the
-selected set against the oracle's (differences allowed only within 1e-3 of
-the k-th score), the attention output against the oracle re-run on the
-GPU's own selection, and the unit calls (indexer, top-k) on the same rows.
+benchmark times; the oracle checks every query row of the two decode
+workloads and of the tiny prefill, and for the long prefills 64 evenly
+spaced rows plus the rows on both sides of every slab boundary of
+dsa_forward, the rows at t = k-1 and t = k, the last row and the planted
+needles: the selected set against the oracle's (differences allowed only
+within 1e-3 of the k-th score), the attention output against the oracle
+re-run on the GPU's own selection, and the unit calls (indexer, top-k) on
+the same rows.
 """
+import types
+
 import numpy as np
 import pytest
 import torch
@@ -17,20 +22,47 @@ import workloads
 from dsa_testutil import (Dev, assert_attn_close, assert_scores_close, assert_selection_ok,
                           ref_attn, ref_scores)
 
-pytestmark = pytest.mark.gpu
+# None: every query row
+SAMPLES = {1: None, 2: 64, 3: None, 4: 64, 5: None, 6: 64}
 
-SAMPLES = {1: None, 2: 12, 3: 8, 4: 8, 5: 4, 6: 8}
+# dsa_forward runs query rows in slabs holding at most 1 GiB of fp32 scores
+# at max_len per row (include/dsa.h); a slab starts at a multiple of this.
+SLAB_SCORE_BYTES = 1 << 30
+
+
+def slab_boundary_rows(n_q, max_len):
+    """The last row of every slab and the first row of the next."""
+    slab = max(1, SLAB_SCORE_BYTES // (4 * max_len))
+    out = []
+    for r0 in range(slab, n_q, slab):
+        out += [r0 - 1, r0]
+    return out
 
 
 def _rows(wl, n):
     if n is None:
         return np.arange(wl.n_q)
-    must = [0, wl.cfg.k - 1, wl.cfg.k, wl.n_q - 1] if wl.cfg.mode == "prefill" else [0, wl.n_q - 1]
+    must = [0, wl.n_q - 1] + slab_boundary_rows(wl.n_q, wl.max_len)
+    if wl.cfg.mode == "prefill":
+        must += [wl.cfg.k - 1, wl.cfg.k]  # t = k-1 (every candidate kept), t = k (one dropped)
     if wl.cfg.plant == "needles":
         must += [t for t, _ in wl.planted]
     return workloads.sample_rows(wl.n_q, n, must)
 
 
+@pytest.mark.parametrize("cid", [4, 6])
+def test_sampled_rows_cover_slab_boundaries(cid):
+    cfg = workloads.config(cid)
+    n_q = sum(cfg.chunks) if cfg.chunks else sum(cfg.lens)
+    wl = types.SimpleNamespace(cfg=cfg, n_q=n_q, max_len=max(cfg.lens), planted=[])
+    rows = set(_rows(wl, SAMPLES[cid]).tolist())
+    assert {4095, 4096, n_q - 4097, n_q - 4096, n_q - 1} <= rows
+    assert len(rows) >= 64 + 2 * (n_q // 4096 - 1)
+    if cfg.mode == "prefill":
+        assert {2047, 2048} <= rows
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("cid", [1, 2, 3, 4, 5, 6])
 def test_forward_matches_oracle(cid):
     wl = workloads.generate(cid)
