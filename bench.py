@@ -170,7 +170,7 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- device run
-def run_device(cid, steps, warmup, rank, world, do_e2e=True):
+def run_device(cid, steps, warmup, rank, world, do_e2e=True, index_reuse=1):
     import sparse_attention_relu_b200 as dsa
 
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -236,7 +236,69 @@ def run_device(cid, steps, warmup, rank, world, do_e2e=True):
     e2e = None
     if do_e2e:
         e2e = run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream)
-    return wl, ms, stage_ms, launches, clocks, e2e
+    reuse = None
+    if index_reuse > 1:
+        reuse = run_index_reuse(dsa, wl, lay, args, out, lse, ws, flush, stream, steps, warmup,
+                                index_reuse, world)
+    return wl, ms, stage_ms, launches, clocks, e2e, reuse
+
+
+def run_index_reuse(dsa, wl, lay, args, out, lse, ws, flush, stream, steps, warmup, layers,
+                    world):
+    """IndexCache ("Linear and Sparse Attention", GLM 5.2 / IndexCache
+    passage): one indexer serves `layers` attention layers.  A step is
+    dsa_forward on layer 1 (indexer, top-k, attention; the indices kept in
+    idx_out), then dsa_sparse_mla_attn on each later layer's own absorbed
+    queries and MLA cache with those indices.  The later layers' inputs are
+    drawn on the device (seeded, the workload's shapes and distribution:
+    N(0, 1/D_K) rounded to bf16); timing as for the main step."""
+    c = wl.cfg
+    dev = out.device
+    idx = torch.empty(wl.n_q, c.k, dtype=torch.int32, device=dev)
+    g = torch.Generator(device=dev)
+    extra = []
+    for layer in range(2, layers + 1):
+        g.manual_seed(c.seed * 100 + layer)
+        q = (torch.randn(wl.n_q, c.H, c.D_K, generator=g, device=dev) * c.mla_std).to(
+            torch.bfloat16)
+        kv = (torch.randn(wl.n_k, c.D_K, generator=g, device=dev) * c.mla_std).to(torch.bfloat16)
+        extra.append((q, kv))
+    nws = dsa.dsa_sparse_mla_attn_workspace_size(lay, c.k, c.H, c.D_K, c.D_V)
+    aws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+    o2 = torch.empty_like(out)
+    l2 = torch.empty_like(lse)
+
+    def step(ev_mid):
+        dsa.dsa_forward(lay, args, out, lse, idx, ws)
+        ev_mid.record(stream)
+        for q, kv in extra:
+            dsa.dsa_sparse_mla_attn(lay, q, kv, idx, c.k, c.D_V, c.sm_scale, o2, l2, aws)
+
+    for _ in range(warmup):
+        step(torch.cuda.Event())
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    first, total = [], []
+    for i in range(steps):
+        flush.fill_(float(i))
+        flush[: 64 << 20].sum()
+        torch.cuda._sleep(SPIN_CYCLES)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        step(e1)
+        e2.record(stream)
+        e2.synchronize()
+        first.append(e0.elapsed_time(e1))
+        total.append(e0.elapsed_time(e2))
+    if world > 1:
+        torch.distributed.barrier()
+    st = dsa.dsa_device_status()
+    if st != dsa.DSA_OK:
+        raise RuntimeError(f"device status after index reuse: {dsa.dsa_status_string(st)}")
+    ms, ms1 = sum(total) / steps, sum(first) / steps
+    return {"layers": layers, "ms_per_step": ms, "layer1_ms": ms1,
+            "later_layer_ms": (ms - ms1) / (layers - 1)}
 
 
 def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
@@ -490,6 +552,15 @@ def run_reference(cid, steps, warmup, n_gpus):
     print(json.dumps(line), flush=True)
 
 
+def _reuse_line(r, ms_max, tokens, world):
+    return {"layers": r["layers"], "value": round(job_throughput(tokens, ms_max, world), 1),
+            "unit": "tokens/s (all layers of the step)", "ms_per_step": round(ms_max, 4),
+            "layer1_ms": round(r["layer1_ms"], 4),
+            "later_layer_ms": round(r["later_layer_ms"], 4),
+            "note": "layer 1: dsa_forward (indexer, top-k, attention); layers 2..L: "
+                    "dsa_sparse_mla_attn on their own q and MLA cache with layer 1's indices"}
+
+
 # --------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -501,6 +572,9 @@ def main():
     ap.add_argument("--decode-workload", default="decode64k", choices=list(WORKLOADS) + ["none"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--index-reuse", type=int, default=1,
+                    help="L > 1 adds an `index_reuse` object: one indexer serving L attention "
+                         "layers (IndexCache), tokens/s of the L-layer step")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -522,18 +596,20 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     peaks = load_peaks()
-    wl, ms, stage_ms, launches, clocks, e2e = run_device(cid, a.steps, a.warmup, rank, world,
-                                                         not a.no_e2e)
+    wl, ms, stage_ms, launches, clocks, e2e, reuse = run_device(
+        cid, a.steps, a.warmup, rank, world, not a.no_e2e, a.index_reuse)
     dec = None
     if a.decode_workload != "none":
         dcid = WORKLOADS[a.decode_workload]
-        dwl, dms, dstage, dlaunch, _, de2e = run_device(dcid, a.steps, a.warmup, rank, world,
-                                                        not a.no_e2e)
-        dec = (dwl, dms, dstage, dlaunch, de2e)
+        dwl, dms, dstage, dlaunch, _, de2e, dreuse = run_device(
+            dcid, a.steps, a.warmup, rank, world, not a.no_e2e, a.index_reuse)
+        dec = (dwl, dms, dstage, dlaunch, de2e, dreuse)
 
     ms = max_over_ranks(ms, world, "cuda")
     e2e_ms = max_over_ranks(e2e["ms_per_step"], world, "cuda") if e2e else None
+    reuse_ms = max_over_ranks(reuse["ms_per_step"], world, "cuda") if reuse else None
     if dec:
+        dreuse_ms = max_over_ranks(dec[5]["ms_per_step"], world, "cuda") if dec[5] else None
         dms = max_over_ranks(dec[1], world, "cuda")
         de2e_ms = max_over_ranks(dec[4]["ms_per_step"], world, "cuda") if dec[4] else None
     tokens = wl.n_q
@@ -559,6 +635,8 @@ def main():
                            "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                            "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
                            "inputs": e2e["inputs"]}
+        if reuse:
+            line["index_reuse"] = _reuse_line(reuse, reuse_ms, tokens, world)
         if clocks:
             line["clocks"] = clocks
         if dec:
@@ -569,6 +647,8 @@ def main():
                               "unit": "tokens/s", "ms_per_step": round(dms, 4),
                               "roofline": droof, "stage_share": dshares,
                               "gpu_launches": dec[3]}
+            if dec[5]:
+                line["decode"]["index_reuse"] = _reuse_line(dec[5], dreuse_ms, dwl.n_q, world)
             if dec[4]:
                 line["decode"]["e2e"] = {
                     "value": round(job_throughput(dwl.n_q, de2e_ms, world), 1), "unit": "tokens/s",
