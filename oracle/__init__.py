@@ -62,6 +62,10 @@ def _load():
         lib.oracle_topk_f64.argtypes = [I64, P, I64, P, I, P]
         lib.oracle_sparse_mla_attn.argtypes = [I64, P, P, P, I, I, I, I, ctypes.c_double, P, P, P, P]
         lib.oracle_dense_mla_attn.argtypes = [I64, P, P, P, I, I, I, ctypes.c_double, P, P, P, P]
+        lib.oracle_sparse_mla_attn_kv.argtypes = [I64, P, P, P, I, I, I, I, ctypes.c_double, P, P,
+                                                  I, P, P, P]
+        lib.oracle_dense_mla_attn_kv.argtypes = [I64, P, P, P, I, I, I, ctypes.c_double, P, P, I,
+                                                 P, P, P]
         _lib = lib
     return _lib
 
@@ -141,8 +145,9 @@ def topk(scores, n_valid, k):
     return out
 
 
-def sparse_mla_attn(qrow, kbase, idx, q, kv, *, D_V, sm_scale):
-    """(out [n, H, D_V], lse [n, H]) fp64; q: uint16 [n_q, H, D_K], kv: uint16 [N_k, D_K]."""
+def sparse_mla_attn(qrow, kbase, idx, q, kv, *, D_V, sm_scale, kv_scale=None):
+    """(out [n, H, D_V], lse [n, H]) fp64; q: uint16 [n_q, H, D_K] (bf16 bits);
+    kv: uint16 [N_k, D_K] bf16 bits, or uint8 e4m3 codes with kv_scale [N_k]."""
     lib = _load()
     _, H, D_K = q.shape
     qrow, pq = _c(qrow, np.int64)
@@ -150,16 +155,17 @@ def sparse_mla_attn(qrow, kbase, idx, q, kv, *, D_V, sm_scale):
     idx, pi = _c(idx, np.int32)
     q, pqq = _raw(q)
     kv, pkv = _raw(kv)
+    kdt, ks, pks = _cache(kv, kv_scale)
     n, k = idx.shape
     out = np.empty((n, H, D_V), np.float64)
     lse = np.empty((n, H), np.float64)
-    lib.oracle_sparse_mla_attn(n, pq, pk, pi, k, H, D_K, D_V, float(sm_scale), pqq, pkv,
-                               out.ctypes.data_as(ctypes.c_void_p),
-                               lse.ctypes.data_as(ctypes.c_void_p))
+    lib.oracle_sparse_mla_attn_kv(n, pq, pk, pi, k, H, D_K, D_V, float(sm_scale), pqq, pkv, kdt,
+                                  pks, out.ctypes.data_as(ctypes.c_void_p),
+                                  lse.ctypes.data_as(ctypes.c_void_p))
     return out, lse
 
 
-def dense_mla_attn(qrow, kbase, tpos, q, kv, *, D_V, sm_scale):
+def dense_mla_attn(qrow, kbase, tpos, q, kv, *, D_V, sm_scale, kv_scale=None):
     """Dense causal attention over positions 0..tpos[i]; same shapes as sparse."""
     lib = _load()
     _, H, D_K = q.shape
@@ -168,10 +174,23 @@ def dense_mla_attn(qrow, kbase, tpos, q, kv, *, D_V, sm_scale):
     tpos, pt = _c(tpos, np.int64)
     q, pqq = _raw(q)
     kv, pkv = _raw(kv)
+    kdt, ks, pks = _cache(kv, kv_scale)
     n = len(qrow)
     out = np.empty((n, H, D_V), np.float64)
     lse = np.empty((n, H), np.float64)
-    lib.oracle_dense_mla_attn(n, pq, pk, pt, H, D_K, D_V, float(sm_scale), pqq, pkv,
-                              out.ctypes.data_as(ctypes.c_void_p),
-                              lse.ctypes.data_as(ctypes.c_void_p))
+    lib.oracle_dense_mla_attn_kv(n, pq, pk, pt, H, D_K, D_V, float(sm_scale), pqq, pkv, kdt, pks,
+                                 out.ctypes.data_as(ctypes.c_void_p),
+                                 lse.ctypes.data_as(ctypes.c_void_p))
     return out, lse
+
+
+def _cache(kv, kv_scale):
+    """Storage type code of the MLA cache and its scale array (e4m3 only)."""
+    if kv.dtype == np.uint8:
+        if kv_scale is None:
+            raise ValueError("an e4m3 cache needs its per-token kv_scale")
+        ks, pks = _c(kv_scale, np.float32)
+        return E4M3, ks, pks
+    if kv.dtype != np.uint16 or kv_scale is not None:
+        raise ValueError("the cache is bf16 bits (uint16) or e4m3 codes (uint8) with kv_scale")
+    return BF16, None, None

@@ -220,19 +220,29 @@ void oracle_topk_f64(int64_t n_rows, const double* scores, int64_t ld, const int
  *   lse[h]  = log sum_s exp(z_s)
  * Positions listed as -1 are empty slots.  With no position at all the
  * output is 0 and lse is -inf.
+ * The cache C is stored as bf16, or as fp8 e4m3 codes with one fp32 scale per
+ * token (the FP8 argument of "GLM sparse attention", ReLU paragraph, read as
+ * applying to the cached latent as it does to the indexer keys): every
+ * element is decoded exactly, C[s, d] = code * kv_scale[s], in fp64.
  */
-static void attend_row(const uint16_t* q, const uint16_t* kv, int64_t kb, const int64_t* pos,
-                       int64_t npos, int H, int D_K, int D_V, double sm_scale, double* out,
-                       double* lse) {
+static double cache_elem(const void* kv, int kv_dtype, const float* kv_scale, int64_t row,
+                         int D_K, int d) {
+  const double x = load_elem(kv, kv_dtype, row * D_K + d);
+  return kv_scale ? x * (double)kv_scale[row] : x;
+}
+
+static void attend_row(const uint16_t* q, const void* kv, int kv_dtype, const float* kv_scale,
+                       int64_t kb, const int64_t* pos, int64_t npos, int H, int D_K, int D_V,
+                       double sm_scale, double* out, double* lse) {
   double* z = (double*)malloc(sizeof(double) * (size_t)(npos > 0 ? npos : 1));
   double* qh = (double*)malloc(sizeof(double) * (size_t)D_K);
   for (int h = 0; h < H; ++h) {
     for (int d = 0; d < D_K; ++d) qh[d] = oracle_bf16_to_f64(q[(int64_t)h * D_K + d]);
     double m = -INFINITY;
     for (int64_t r = 0; r < npos; ++r) {
-      const uint16_t* c = kv + (kb + pos[r]) * D_K;
       double dot = 0.0;
-      for (int d = 0; d < D_K; ++d) dot += qh[d] * oracle_bf16_to_f64(c[d]);
+      for (int d = 0; d < D_K; ++d)
+        dot += qh[d] * cache_elem(kv, kv_dtype, kv_scale, kb + pos[r], D_K, d);
       z[r] = sm_scale * dot;
       if (z[r] > m) m = z[r];
     }
@@ -246,8 +256,8 @@ static void attend_row(const uint16_t* q, const uint16_t* kv, int64_t kb, const 
     for (int64_t r = 0; r < npos; ++r) {
       double p = exp(z[r] - m);
       sum += p;
-      const uint16_t* c = kv + (kb + pos[r]) * D_K;
-      for (int v = 0; v < D_V; ++v) o[v] += p * oracle_bf16_to_f64(c[v]);
+      for (int v = 0; v < D_V; ++v)
+        o[v] += p * cache_elem(kv, kv_dtype, kv_scale, kb + pos[r], D_K, v);
     }
     for (int v = 0; v < D_V; ++v) o[v] /= sum;
     lse[h] = m + log(sum);
@@ -259,35 +269,52 @@ static void attend_row(const uint16_t* q, const uint16_t* kv, int64_t kb, const 
 /*
  * Sparse MLA attention: row i attends over the positions idx[i, 0:k] (local
  * to its sequence, -1 = empty) of the cache rows starting at kbase[i].
- * q: bf16 [*, H, D_K] addressed by qrow[i]; kv: bf16 [N_k, D_K].
+ * q: bf16 [*, H, D_K] addressed by qrow[i]; kv: [N_k, D_K] in kv_dtype (bf16,
+ * or e4m3 with kv_scale [N_k]; kv_scale NULL for bf16).
  * out: [n_rows, H, D_V]; lse: [n_rows, H].
  */
-void oracle_sparse_mla_attn(int64_t n_rows, const int64_t* qrow, const int64_t* kbase,
-                            const int32_t* idx, int k, int H, int D_K, int D_V, double sm_scale,
-                            const uint16_t* q, const uint16_t* kv, double* out, double* lse) {
+void oracle_sparse_mla_attn_kv(int64_t n_rows, const int64_t* qrow, const int64_t* kbase,
+                               const int32_t* idx, int k, int H, int D_K, int D_V,
+                               double sm_scale, const uint16_t* q, const void* kv, int kv_dtype,
+                               const float* kv_scale, double* out, double* lse) {
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t i = 0; i < n_rows; ++i) {
     int64_t* pos = (int64_t*)malloc(sizeof(int64_t) * (size_t)(k > 0 ? k : 1));
     int64_t np = 0;
     for (int r = 0; r < k; ++r)
       if (idx[i * (int64_t)k + r] >= 0) pos[np++] = idx[i * (int64_t)k + r];
-    attend_row(q + qrow[i] * (int64_t)H * D_K, kv, kbase[i], pos, np, H, D_K, D_V, sm_scale,
-               out + i * (int64_t)H * D_V, lse + i * (int64_t)H);
+    attend_row(q + qrow[i] * (int64_t)H * D_K, kv, kv_dtype, kv_scale, kbase[i], pos, np, H, D_K,
+               D_V, sm_scale, out + i * (int64_t)H * D_V, lse + i * (int64_t)H);
     free(pos);
   }
 }
 
+void oracle_sparse_mla_attn(int64_t n_rows, const int64_t* qrow, const int64_t* kbase,
+                            const int32_t* idx, int k, int H, int D_K, int D_V, double sm_scale,
+                            const uint16_t* q, const uint16_t* kv, double* out, double* lse) {
+  oracle_sparse_mla_attn_kv(n_rows, qrow, kbase, idx, k, H, D_K, D_V, sm_scale, q, kv, OR_BF16,
+                            NULL, out, lse);
+}
+
 /* Dense causal MLA attention of row i over every position 0..tpos[i]. */
-void oracle_dense_mla_attn(int64_t n_rows, const int64_t* qrow, const int64_t* kbase,
-                           const int64_t* tpos, int H, int D_K, int D_V, double sm_scale,
-                           const uint16_t* q, const uint16_t* kv, double* out, double* lse) {
+void oracle_dense_mla_attn_kv(int64_t n_rows, const int64_t* qrow, const int64_t* kbase,
+                              const int64_t* tpos, int H, int D_K, int D_V, double sm_scale,
+                              const uint16_t* q, const void* kv, int kv_dtype,
+                              const float* kv_scale, double* out, double* lse) {
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t i = 0; i < n_rows; ++i) {
     int64_t n = tpos[i] + 1;
     int64_t* pos = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n > 0 ? n : 1));
     for (int64_t s = 0; s < n; ++s) pos[s] = s;
-    attend_row(q + qrow[i] * (int64_t)H * D_K, kv, kbase[i], pos, n, H, D_K, D_V, sm_scale,
-               out + i * (int64_t)H * D_V, lse + i * (int64_t)H);
+    attend_row(q + qrow[i] * (int64_t)H * D_K, kv, kv_dtype, kv_scale, kbase[i], pos, n, H, D_K,
+               D_V, sm_scale, out + i * (int64_t)H * D_V, lse + i * (int64_t)H);
     free(pos);
   }
+}
+
+void oracle_dense_mla_attn(int64_t n_rows, const int64_t* qrow, const int64_t* kbase,
+                           const int64_t* tpos, int H, int D_K, int D_V, double sm_scale,
+                           const uint16_t* q, const uint16_t* kv, double* out, double* lse) {
+  oracle_dense_mla_attn_kv(n_rows, qrow, kbase, tpos, H, D_K, D_V, sm_scale, q, kv, OR_BF16, NULL,
+                           out, lse);
 }

@@ -81,7 +81,8 @@ def ref_scores(wl, rows, with_abs=True):
 def ref_attn(wl, rows, idx_rows):
     c = wl.cfg
     return oracle.sparse_mla_attn(wl.qrow[rows], wl.kbase[rows], idx_rows, wl.raw(wl.q),
-                                  wl.raw(wl.kv), D_V=c.D_V, sm_scale=c.sm_scale)
+                                  wl.raw(wl.kv), D_V=c.D_V, sm_scale=c.sm_scale,
+                                  kv_scale=wl.raw(getattr(wl, "kv_scale", None)))
 
 
 def assert_scores_close(got, ref, A, tpos):

@@ -382,6 +382,77 @@ def test_full_selection_equals_dense(oracle_mod):
     assert np.allclose(o_s, o_d, rtol=1e-12, atol=1e-15) and np.allclose(l_s, l_d, rtol=1e-13)
 
 
+def _e4m3_cache(rng, N_k, D_K, pow2=False):
+    """e4m3 codes [N_k, D_K] (uint8, never the NaN code) and per-token scales."""
+    x = torch.from_numpy(rng.standard_normal((N_k, D_K)) / math.sqrt(D_K) * 8)
+    codes, scale = workloads.quantize_e4m3_per_token(x.float())
+    if pow2:  # scales that are powers of two: code * scale is exact in bf16
+        scale = torch.exp2(torch.round(torch.log2(scale)))
+    return codes.view(torch.uint8).numpy(), scale.numpy()
+
+
+def test_fp8_cache_attn_matches_sdpa_on_decoded_values(oracle_mod):
+    """FP8 MLA cache (e4m3 codes, one fp32 scale per token): the oracle's
+    attention equals torch SDPA in fp64 on the decoded cache, table[code] *
+    scale, with the selection as a mask; the value is the first D_V decoded
+    columns.  The decode table is pinned to torch's own e4m3 cast above."""
+    rng = np.random.default_rng(21)
+    H, D_K, D_V, L, k = 4, 80, 64, 60, 15
+    qb, qf, _, _ = _mla_inputs(rng, 3, H, D_K, L)
+    codes, scale = _e4m3_cache(rng, L, D_K)
+    table = torch.tensor([0.0] * 256, dtype=torch.float64)
+    table[:] = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).double()
+    cf = (table[torch.from_numpy(codes).long()] * torch.from_numpy(scale).double()[:, None]).numpy()
+    idx = np.full((3, k), -1, np.int32)
+    for i in range(3):
+        idx[i, rng.permutation(k)[: k - 2 * i]] = rng.choice(L, size=k - 2 * i, replace=False)
+    sc = 1 / math.sqrt(D_K)
+    out, lse = oracle_mod.sparse_mla_attn(np.arange(3), np.zeros(3, np.int64), idx, qb, codes,
+                                          D_V=D_V, sm_scale=sc, kv_scale=scale)
+    for i in range(3):
+        mask = np.zeros((H, L), bool)
+        mask[:, idx[i][idx[i] >= 0]] = True
+        ref = _sdpa(qf[i], cf, cf[:, :D_V].copy(), sc, mask)
+        assert np.allclose(out[i], ref, rtol=1e-12, atol=1e-14)
+        z = torch.from_numpy(qf[i] @ cf[idx[i][idx[i] >= 0]].T * sc)
+        assert np.allclose(lse[i], torch.logsumexp(z, dim=1).numpy(), rtol=1e-13, atol=1e-13)
+    # a single selected token: the output is its decoded latent exactly
+    one = np.array([[-1, 7, -1]], np.int32)
+    o1, l1 = oracle_mod.sparse_mla_attn([0], [0], one, qb, codes, D_V=D_V, sm_scale=0.5,
+                                        kv_scale=scale)
+    assert np.array_equal(o1[0], np.broadcast_to(cf[7, :D_V], (H, D_V)))
+    # dense over an fp8 cache equals sparse with every position selected
+    T = 20
+    od, ld = oracle_mod.dense_mla_attn(np.arange(T), np.zeros(T, np.int64), np.arange(T), qb[:1]
+                                       .repeat(T, 0), codes, D_V=D_V, sm_scale=sc,
+                                       kv_scale=scale)
+    full = np.where(np.arange(T)[None, :] <= np.arange(T)[:, None], np.arange(T)[None, :], -1)
+    os_, ls_ = oracle_mod.sparse_mla_attn(np.arange(T), np.zeros(T, np.int64),
+                                          full.astype(np.int32), qb[:1].repeat(T, 0), codes,
+                                          D_V=D_V, sm_scale=sc, kv_scale=scale)
+    assert np.allclose(od, os_, rtol=1e-12, atol=1e-15) and np.allclose(ld, ls_, rtol=1e-13)
+
+
+def test_fp8_cache_equals_bf16_cache_when_exact(oracle_mod):
+    """With power-of-two scales every decoded element code * scale is exactly
+    a bf16 value, so the fp8 path must equal the bf16 path on that cache."""
+    rng = np.random.default_rng(22)
+    H, D_K, D_V, L, k = 3, 48, 32, 30, 9
+    qb, _, _, _ = _mla_inputs(rng, 2, H, D_K, L)
+    codes, scale = _e4m3_cache(rng, L, D_K, pow2=True)
+    dec = torch.from_numpy(codes).view(torch.float8_e4m3fn).float() * torch.from_numpy(scale)[:, None]
+    cb = dec.to(torch.bfloat16)
+    assert torch.equal(cb.float(), dec)  # exact
+    cbits = cb.view(torch.int16).numpy().view(np.uint16)
+    idx = np.stack([rng.choice(L, size=k, replace=False) for _ in range(2)]).astype(np.int32)
+    a = oracle_mod.sparse_mla_attn([0, 1], [0, 0], idx, qb, codes, D_V=D_V, sm_scale=0.4,
+                                   kv_scale=scale)
+    b = oracle_mod.sparse_mla_attn([0, 1], [0, 0], idx, qb, cbits, D_V=D_V, sm_scale=0.4)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    with pytest.raises(ValueError):
+        oracle_mod.sparse_mla_attn([0], [0], idx[:1], qb, codes, D_V=D_V, sm_scale=0.4)
+
+
 # ---------------------------------------------------------------- workloads
 @pytest.mark.slow
 def test_config2_needles_rank_first(oracle_mod):

@@ -58,6 +58,7 @@ class Config:
     alpha: float = 64.0
     seed: int = 0
     chunks: Optional[List[int]] = None  # chunked: new query tokens per sequence (<= its length)
+    kv_dtype: str = "bf16"  # MLA cache storage: "bf16" | "e4m3" (codes + one fp32 scale per token)
 
     def __post_init__(self):
         if not self.seed:
@@ -96,7 +97,7 @@ def config(cid: int) -> Config:
 
 def custom(mode="prefill", lens=(300,), H_I=64, D_I=128, idx_dtype="bf16", k=64, H=128,
            D_K=576, D_V=512, sm_scale=None, w_std=None, mla_std=None, plant=None, seed=7,
-           name=None, chunks=None) -> Config:
+           name=None, chunks=None, kv_dtype="bf16") -> Config:
     """A small workload with the structure of the big ones (tests).  For
     mode "chunked", chunks[b] new query tokens close sequence b."""
     lens = list(lens)
@@ -105,7 +106,7 @@ def custom(mode="prefill", lens=(300,), H_I=64, D_I=128, idx_dtype="bf16", k=64,
                   sm_scale if sm_scale is not None else 1 / math.sqrt(D_K),
                   w_std if w_std is not None else 1 / math.sqrt(H_I),
                   mla_std if mla_std is not None else 1 / math.sqrt(D_K), plant=plant, seed=seed,
-                  chunks=list(chunks) if chunks is not None else None)
+                  chunks=list(chunks) if chunks is not None else None, kv_dtype=kv_dtype)
 
 
 def _seed(*parts) -> int:
@@ -145,7 +146,8 @@ class Workload:
 
     kv_offsets int32 [B+1]; q_idx [n_q, H_I, D_I]; q_scale fp32 [n_q, H_I] or
     None; w fp32 [n_q, H_I]; k_idx [N_k, D_I]; k_scale fp32 [N_k] or None;
-    q bf16 [n_q, H, D_K]; kv bf16 [N_k, D_K].
+    q bf16 [n_q, H, D_K]; kv bf16 [N_k, D_K], or (cfg.kv_dtype "e4m3") fp8 codes
+    [N_k, D_K] with kv_scale fp32 [N_k].
     Query row r belongs to sequence seq[r] at local position tpos[r]; its keys
     are rows kv_offsets[seq] ... kv_offsets[seq] + tpos[r].
     """
@@ -216,10 +218,23 @@ class Workload:
             rows_per_block = max(1, (1 << 24) // (cfg.H * cfg.D_K))
             self.q = _normal_blocks(seed, "q", (self.n_q, cfg.H, cfg.D_K), cfg.mla_std,
                                     torch.bfloat16, rows_per_block, pin)
-            self.kv = _normal_blocks(seed, "kv", (self.n_k, cfg.D_K), cfg.mla_std,
-                                     torch.bfloat16, max(1, (1 << 24) // cfg.D_K), pin)
+            kv_rows = max(1, (1 << 24) // cfg.D_K)
+            self.kv_scale = None
+            if cfg.kv_dtype == "bf16":
+                self.kv = _normal_blocks(seed, "kv", (self.n_k, cfg.D_K), cfg.mla_std,
+                                         torch.bfloat16, kv_rows, pin)
+            elif cfg.kv_dtype == "e4m3":
+                # the same fp32 draws as the bf16 cache, quantised per token
+                kv32 = _normal_blocks(seed, "kv", (self.n_k, cfg.D_K), cfg.mla_std,
+                                      torch.float32, kv_rows)
+                self.kv, self.kv_scale = quantize_e4m3_per_token(kv32)
+                del kv32
+                if pin:
+                    self.kv, self.kv_scale = self.kv.pin_memory(), self.kv_scale.pin_memory()
+            else:
+                raise ValueError(cfg.kv_dtype)
         else:
-            self.q = self.kv = None
+            self.q = self.kv = self.kv_scale = None
 
     # -- planted structure -------------------------------------------------
     def _direction(self, qI, r):
@@ -266,7 +281,7 @@ class Workload:
         other = object.__new__(Workload)
         other.__dict__.update(self.__dict__)
         for name in ("q_idx", "k_idx", "w", "q_scale", "k_scale", "kv_offsets", "q_offsets", "q",
-                     "kv"):
+                     "kv", "kv_scale"):
             t = getattr(self, name)
             if t is not None:
                 setattr(other, name, t.to(device, non_blocking=True))
