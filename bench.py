@@ -82,8 +82,8 @@ def algorithmic_work(wl):
     indexer: 2*H_I*D_I flop per causal (t, s) pair; key bytes D_I*esize
              (+4 for an fp8 scale) per key a decode row scans;
     top-k:   4 B read per candidate + 4k B written per row;
-    attention: H*(2*D_K + 2*D_V) flop and D_K*2 gathered bytes per
-             (row, selected position).
+    attention: H*(2*D_K + 2*D_V) flop and D_K*2 gathered bytes (D_K + 4 for
+             an e4m3 cache with its scale) per (row, selected position).
     """
     c = wl.cfg
     n = (wl.tpos + 1).astype(np.float64)
@@ -94,9 +94,14 @@ def algorithmic_work(wl):
         "idx_bytes": n * (c.D_I * esz + (4 if c.idx_dtype == "e4m3" else 0)),
         "topk_bytes": 4.0 * n + 4.0 * c.k,
         "attn_flop": c.H * (2.0 * c.D_K + 2.0 * c.D_V) * sel,
-        "attn_bytes": 2.0 * c.D_K * sel,
+        # gathered bytes per selected token: a bf16 row, or e4m3 codes + a fp32 scale
+        "attn_bytes": (2.0 * c.D_K if c.kv_dtype == "bf16" else c.D_K + 4.0) * sel,
     }
 
+
+# decode end to end: rows per slab of dsa_forward_host (the copies of one slab
+# overlap the kernels of another)
+DECODE_SLAB_ROWS = 16
 
 SPIN_CYCLES = 1_000_000  # about 0.5 ms at 1.9-2 GHz, longer than the host takes to queue a step
 
@@ -170,17 +175,31 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- device run
-def run_device(cid, steps, warmup, rank, world, do_e2e=True, index_reuse=1):
+def workload_config(cid, kv_dtype="bf16"):
+    cfg = workloads.config(cid)
+    if kv_dtype != "bf16":
+        cfg.kv_dtype = kv_dtype
+    return cfg
+
+
+def describe(cfg):
+    d = DESCR[cfg.cid]
+    if cfg.kv_dtype == "e4m3":
+        d = d.replace("576/512 bf16", "576/512, FP8 e4m3 MLA cache with per-token fp32 scales")
+    return d
+
+
+def run_device(cid, steps, warmup, rank, world, do_e2e=True, index_reuse=1, kv_dtype="bf16"):
     import sparse_attention_relu_b200 as dsa
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    wl = workloads.generate(cid, pin=do_e2e)
+    wl = workloads.generate(workload_config(cid, kv_dtype), pin=do_e2e)
     c = wl.cfg
     d = wl.to(dev)
     lay = dsa.Layout.of(wl, d.kv_offsets, d.q_offsets)
     args = dsa.forward_args(q_idx=d.q_idx, q_scale=d.q_scale, w=d.w, k_idx=d.k_idx,
                             k_scale=d.k_scale, q=d.q, kv=d.kv, D_V=c.D_V, sm_scale=c.sm_scale,
-                            k=c.k)
+                            k=c.k, kv_scale=d.kv_scale)
     nws = dsa.dsa_forward_workspace_size(lay, args)
     ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
     out = torch.empty(wl.n_q, c.H, c.D_V, dtype=torch.bfloat16, device=dev)
@@ -261,8 +280,12 @@ def run_index_reuse(dsa, wl, lay, args, out, lse, ws, flush, stream, steps, warm
         g.manual_seed(c.seed * 100 + layer)
         q = (torch.randn(wl.n_q, c.H, c.D_K, generator=g, device=dev) * c.mla_std).to(
             torch.bfloat16)
-        kv = (torch.randn(wl.n_k, c.D_K, generator=g, device=dev) * c.mla_std).to(torch.bfloat16)
-        extra.append((q, kv))
+        kv32 = torch.randn(wl.n_k, c.D_K, generator=g, device=dev) * c.mla_std
+        if c.kv_dtype == "e4m3":
+            extra.append((q, *workloads.quantize_e4m3_per_token(kv32)))
+        else:
+            extra.append((q, kv32.to(torch.bfloat16), None))
+        del kv32
     nws = dsa.dsa_sparse_mla_attn_workspace_size(lay, c.k, c.H, c.D_K, c.D_V)
     aws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
     o2 = torch.empty_like(out)
@@ -271,8 +294,12 @@ def run_index_reuse(dsa, wl, lay, args, out, lse, ws, flush, stream, steps, warm
     def step(ev_mid):
         dsa.dsa_forward(lay, args, out, lse, idx, ws)
         ev_mid.record(stream)
-        for q, kv in extra:
-            dsa.dsa_sparse_mla_attn(lay, q, kv, idx, c.k, c.D_V, c.sm_scale, o2, l2, aws)
+        for q, kv, kv_scale in extra:
+            if kv_scale is None:
+                dsa.dsa_sparse_mla_attn(lay, q, kv, idx, c.k, c.D_V, c.sm_scale, o2, l2, aws)
+            else:
+                dsa.dsa_sparse_mla_attn_e4m3(lay, q, kv, kv_scale, idx, c.k, c.D_V, c.sm_scale,
+                                             o2, l2, aws)
 
     for _ in range(warmup):
         step(torch.cuda.Event())
@@ -311,9 +338,10 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
     untimed); a step's inputs are the new queries and the cache rows of the
     new tokens (indexer key, its scale, latent + rotary row: one per sequence
     in decode, the chunk's in chunked prefill), written in place every step."""
-    names = ["q_idx", "q_scale", "w", "k_idx", "k_scale", "q", "kv", "kv_offsets", "q_offsets"]
+    names = ["q_idx", "q_scale", "w", "k_idx", "k_scale", "q", "kv", "kv_scale", "kv_offsets",
+             "q_offsets"]
     resident = c.mode in ("decode", "chunked")
-    cache = ("k_idx", "k_scale", "kv") if resident else ()
+    cache = ("k_idx", "k_scale", "kv", "kv_scale") if resident else ()
     host = {n: getattr(wl, n) for n in names if getattr(wl, n) is not None}
     dbuf = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
     for n in cache + ("kv_offsets", "q_offsets") if resident else ():
@@ -342,19 +370,23 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
     lay2 = dsa.Layout.of(wl, dbuf["kv_offsets"], dbuf.get("q_offsets"))
     args = dsa.forward_args(q_idx=dbuf["q_idx"], q_scale=dbuf.get("q_scale"), w=dbuf["w"],
                             k_idx=dbuf["k_idx"], k_scale=dbuf.get("k_scale"), q=dbuf["q"],
-                            kv=dbuf["kv"], D_V=c.D_V, sm_scale=c.sm_scale, k=c.k)
+                            kv=dbuf["kv"], D_V=c.D_V, sm_scale=c.sm_scale, k=c.k,
+                            kv_scale=dbuf.get("kv_scale"))
     out = torch.empty(wl.n_q, c.H, c.D_V, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(wl.n_q, c.H, dtype=torch.float32, device=dev)
-    # prefill and chunked prefill run several slabs: dsa_forward_host overlaps
-    # the query uploads, the kernels and the output downloads slab by slab (a
-    # resident cache is passed as NULL on the host side); decode is one slab
-    use_host = c.mode != "decode"
+    # dsa_forward_host overlaps the query uploads, the kernels and the output
+    # downloads slab by slab (a resident cache is passed as NULL on the host
+    # side); decode rows run in slabs of DECODE_SLAB_ROWS so that its copies
+    # overlap too
+    use_host = True
+    slab_cap = DECODE_SLAB_ROWS if c.mode == "decode" else 0
     if use_host:
         hargs = dsa.forward_args(q_idx=host["q_idx"], q_scale=host.get("q_scale"), w=host["w"],
                                  k_idx=host.get("k_idx"), k_scale=host.get("k_scale"),
                                  q=host["q"], kv=host.get("kv"), D_V=c.D_V, sm_scale=c.sm_scale,
-                                 k=c.k, host=True)
-        nws = dsa.dsa_forward_host_workspace_size(lay2, args)
+                                 k=c.k, host=True, kv_scale=host.get("kv_scale"),
+                                 kv_dtype=args.kv_dtype)
+        nws = dsa.dsa_forward_host_workspace_size(lay2, args, slab_cap)
         if nws > ws.numel():
             ws = torch.empty(nws, dtype=torch.uint8, device=dev)
 
@@ -369,7 +401,7 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
             else:
                 dbuf[n].index_copy_(0, last_dev, stage)
         if use_host:
-            dsa.dsa_forward_host(lay2, hargs, args, out_h, lse_h, out, lse, ws)
+            dsa.dsa_forward_host(lay2, hargs, args, out_h, lse_h, out, lse, ws, slab_cap)
             return
         dsa.dsa_forward(lay2, args, out, lse, None, ws)
         out_h.copy_(out, non_blocking=True)
@@ -387,7 +419,8 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
     inputs = ("new queries + the new tokens' cache rows per step (caches resident in HBM)"
               if cache else "every input of the step (queries, indexer keys, MLA cache)")
     if use_host:
-        inputs += "; copies overlapped with the kernels slab by slab (dsa_forward_host)"
+        inputs += "; copies overlapped with the kernels slab by slab (dsa_forward_host"
+        inputs += f", {slab_cap} rows per slab)" if slab_cap else ")"
     return {"ms_per_step": ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "inputs": inputs}
 
@@ -491,7 +524,7 @@ def oracle_rows(wl, rows):
                               q_scale=wl.raw(wl.q_scale), k_scale=wl.raw(wl.k_scale))
     idx = oracle.topk(I, wl.tpos[rows] + 1, c.k)
     oracle.sparse_mla_attn(wl.qrow[rows], wl.kbase[rows], idx, wl.raw(wl.q), wl.raw(wl.kv),
-                           D_V=c.D_V, sm_scale=c.sm_scale)
+                           D_V=c.D_V, sm_scale=c.sm_scale, kv_scale=wl.raw(wl.kv_scale))
 
 
 def cpu_baseline(cid, budget_s=20.0, wl=None):
@@ -519,11 +552,11 @@ def cpu_baseline(cid, budget_s=20.0, wl=None):
                       f"(all three stages, fp64), {t_used:.1f} s"}
 
 
-def run_reference(cid, steps, warmup, n_gpus):
+def run_reference(cid, steps, warmup, n_gpus, kv_dtype="bf16"):
     import oracle
 
     oracle.build()
-    wl = workloads.generate(cid)
+    wl = workloads.generate(workload_config(cid, kv_dtype))
     # four rows per oracle thread each step: every core works, and the dynamic
     # row schedule evens out the rows' different causal lengths
     rows_per_step = min(wl.n_q, 4 * oracle.num_threads())
@@ -543,7 +576,7 @@ def run_reference(cid, steps, warmup, n_gpus):
             "n_gpus": n_gpus, "steps": steps, "warmup": warmup,
             "ms_per_step": round(dt / steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": DESCR[cid], "sample_rows_per_step": rows_per_step},
+            "config": {"workload": describe(wl.cfg), "sample_rows_per_step": rows_per_step},
             "cpu_baseline": {"kind": "oracle", "cores": oracle.num_threads(), "value": round(value, 3),
                              "sample": f"{done} evenly spaced query rows over {steps} steps "
                                        f"({rows_per_step} per step, all three stages, fp64)"},
@@ -572,6 +605,9 @@ def main():
     ap.add_argument("--decode-workload", default="decode64k", choices=list(WORKLOADS) + ["none"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-dtype", default="bf16", choices=["bf16", "e4m3"],
+                    help="storage of the MLA cache: bf16, or FP8 e4m3 codes with per-token "
+                         "scales (dsa_sparse_mla_attn_e4m3)")
     ap.add_argument("--index-reuse", type=int, default=1,
                     help="L > 1 adds an `index_reuse` object: one indexer serving L attention "
                          "layers (IndexCache), tokens/s of the L-layer step")
@@ -586,7 +622,7 @@ def main():
 
     if a.impl == "reference":
         if rank == 0:
-            run_reference(cid, a.steps, a.warmup, a.gpus)
+            run_reference(cid, a.steps, a.warmup, a.gpus, a.kv_dtype)
         return
 
     torch.cuda.set_device(local)
@@ -597,12 +633,12 @@ def main():
                                              device_id=torch.device("cuda", local))
     peaks = load_peaks()
     wl, ms, stage_ms, launches, clocks, e2e, reuse = run_device(
-        cid, a.steps, a.warmup, rank, world, not a.no_e2e, a.index_reuse)
+        cid, a.steps, a.warmup, rank, world, not a.no_e2e, a.index_reuse, a.kv_dtype)
     dec = None
     if a.decode_workload != "none":
         dcid = WORKLOADS[a.decode_workload]
         dwl, dms, dstage, dlaunch, _, de2e, dreuse = run_device(
-            dcid, a.steps, a.warmup, rank, world, not a.no_e2e, a.index_reuse)
+            dcid, a.steps, a.warmup, rank, world, not a.no_e2e, a.index_reuse, a.kv_dtype)
         dec = (dwl, dms, dstage, dlaunch, de2e, dreuse)
 
     ms = max_over_ranks(ms, world, "cuda")
@@ -621,9 +657,10 @@ def main():
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": {"f32": "f32", "bf16": "bf16", "e4m3": "e4m3+bf16"}[cfg.idx_dtype],
+            "dtype": {"f32": "f32", "bf16": "bf16", "e4m3": "e4m3+bf16"}[cfg.idx_dtype]
+                     + ("+e4m3 cache" if cfg.kv_dtype == "e4m3" else ""),
             "data": "synthetic",
-            "config": {"workload": DESCR[cid], "tokens_per_step_per_gpu": tokens,
+            "config": {"workload": describe(cfg), "tokens_per_step_per_gpu": tokens,
                        "k": cfg.k, "l2": "flushed before every timed step (512 MB write, 256 MB of it read back)",
                        "queued": "step launches queued behind a 0.5 ms spin kernel outside the timed interval",
                        "parallelism": f"{world} independent replicas (weak scaling)"},
@@ -642,7 +679,7 @@ def main():
         if dec:
             dwl = dec[0]
             droof, dshares = roofline(dwl, dec[2], peaks)
-            line["decode"] = {"workload": DESCR[dwl.cfg.cid],
+            line["decode"] = {"workload": describe(dwl.cfg),
                               "value": round(job_throughput(dwl.n_q, dms, world), 1),
                               "unit": "tokens/s", "ms_per_step": round(dms, 4),
                               "roofline": droof, "stage_share": dshares,

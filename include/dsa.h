@@ -155,9 +155,34 @@ dsa_status_t dsa_sparse_mla_attn(const dsa_layout_t* layout, const void* q, cons
                                  int32_t D_V, float sm_scale, void* out, float* lse,
                                  void* workspace, size_t ws_bytes, void* stream);
 
-/* Workspace bytes dsa_sparse_mla_attn needs for this layout and shape. */
+/* Workspace bytes dsa_sparse_mla_attn (and dsa_sparse_mla_attn_e4m3) need
+ * for this layout and shape. */
 size_t dsa_sparse_mla_attn_workspace_size(const dsa_layout_t* layout, int32_t k, int32_t H,
                                           int32_t D_K, int32_t D_V);
+
+/*
+ * Stage 3 over an FP8 MLA cache.  "GLM sparse attention" (ReLU paragraph)
+ * gives FP8 as the indexer's precision; this call applies the same storage
+ * format to the cached latent + rotary rows, halving the bytes each selected
+ * token costs to gather (576 instead of 1152 at D_K = 576):
+ *
+ *   C[s, d] = code(kv[kbase + s, d]) * kv_scale[kbase + s]
+ *
+ * with code() the exact value of an OCP e4m3 byte, and then exactly the
+ * attention of dsa_sparse_mla_attn on that C (the value is C[s, 0:D_V]).
+ *  kv       [n_k, D_K] e4m3 codes (raw bytes; the NaN codes are not allowed)
+ *  kv_scale [n_k] fp32, one scale per cached token
+ * q, idx, out, lse, workspace and every error: as dsa_sparse_mla_attn; D_K
+ * must be a multiple of 16.  The codes are decoded exactly to bf16 on the
+ * device and the MMAs are the bf16 ones: each score is multiplied by its
+ * token's scale, and the PV operand holds p * scale (rounded to bf16, like p
+ * in dsa_sparse_mla_attn); the softmax denominator sums the fp32 p.
+ */
+dsa_status_t dsa_sparse_mla_attn_e4m3(const dsa_layout_t* layout, const void* q, const void* kv,
+                                      const float* kv_scale, const int32_t* idx, int32_t k,
+                                      int32_t H, int32_t D_K, int32_t D_V, float sm_scale,
+                                      void* out, float* lse, void* workspace, size_t ws_bytes,
+                                      void* stream);
 
 /*
  * dsa_sparse_mla_attn for callers that cannot allocate device memory.
@@ -202,7 +227,10 @@ typedef struct {
   float sm_scale;
   const void* q;
   const void* kv;
-  int32_t k; /* top-k budget */
+  int32_t k;            /* top-k budget */
+  int32_t kv_dtype;     /* DSA_BF16, or DSA_E4M3 (then kv holds codes, see below) */
+  const float* kv_scale; /* DSA_E4M3: [n_k] fp32 per-token cache scales
+                            (dsa_sparse_mla_attn_e4m3); NULL for bf16 */
 } dsa_forward_args_t;
 
 /* Workspace bytes dsa_forward needs (scores slab, indices, attention partials). */
@@ -299,7 +327,8 @@ dsa_status_t dsa_selftest_wait_timeout(int64_t cycles, void* stream);
 /* Static description of a status code. */
 const char* dsa_status_string(dsa_status_t status);
 
-/* ABI version, bumped on any signature change. */
+/* ABI version, bumped on any signature change (4: the FP8 MLA cache, fields
+ * kv_dtype / kv_scale of dsa_forward_args_t). */
 int32_t dsa_abi_version(void);
 
 #ifdef __cplusplus

@@ -48,7 +48,8 @@ class dsa_forward_args_t(ctypes.Structure):
                 ("k_idx", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
                 ("H", ctypes.c_int32), ("D_K", ctypes.c_int32), ("D_V", ctypes.c_int32),
                 ("sm_scale", ctypes.c_float), ("q", ctypes.c_void_p), ("kv", ctypes.c_void_p),
-                ("k", ctypes.c_int32)]
+                ("k", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
+                ("kv_scale", ctypes.c_void_p)]
 
 
 _lib = None
@@ -71,6 +72,8 @@ def lib():
                                           P, SZ, P]
         L.dsa_sparse_mla_attn_noalloc.argtypes = [LP, P, P, P, I32, I32, I32, I32,
                                                   ctypes.c_float, P, P, P]
+        L.dsa_sparse_mla_attn_e4m3.argtypes = [LP, P, P, P, P, I32, I32, I32, I32,
+                                               ctypes.c_float, P, P, P, SZ, P]
         L.dsa_sparse_mla_attn_workspace_size.argtypes = [LP, I32, I32, I32, I32]
         L.dsa_sparse_mla_attn_workspace_size.restype = SZ
         L.dsa_forward_workspace_size.argtypes = [LP, AP]
@@ -86,7 +89,7 @@ def lib():
         L.dsa_status_string.restype = ctypes.c_char_p
         L.dsa_abi_version.restype = I32
         for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn",
-                     "dsa_sparse_mla_attn_noalloc", "dsa_forward",
+                     "dsa_sparse_mla_attn_noalloc", "dsa_sparse_mla_attn_e4m3", "dsa_forward",
                      "dsa_forward_timed", "dsa_forward_host", "dsa_device_status",
                      "dsa_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
@@ -181,6 +184,22 @@ def dsa_sparse_mla_attn(layout: Layout, q, kv, idx, k: int, D_V: int, sm_scale: 
     return out
 
 
+def dsa_sparse_mla_attn_e4m3(layout: Layout, q, kv, kv_scale, idx, k: int, D_V: int,
+                             sm_scale: float, out, lse=None, workspace=None, stream=None):
+    """Stage 3 over an FP8 cache: kv[n_k, D_K] float8_e4m3fn codes with one fp32
+    scale per token (kv_scale[n_k]); out and lse as dsa_sparse_mla_attn."""
+    _, H, D_K = q.shape
+    if kv.dtype != torch.float8_e4m3fn:
+        raise ValueError("dsa_sparse_mla_attn_e4m3 takes a float8_e4m3fn cache")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().dsa_sparse_mla_attn_e4m3(layout.ref, _ptr(q), _ptr(kv), _ptr(kv_scale),
+                                          _ptr(idx), int(k), H, D_K, int(D_V), float(sm_scale),
+                                          _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
+                                          _stream(stream)),
+           "dsa_sparse_mla_attn_e4m3")
+    return out
+
+
 def dsa_sparse_mla_attn_noalloc(layout: Layout, q, kv, idx, k: int, D_V: int, sm_scale: float,
                                 out, lse=None, stream=None):
     """Stage 3 without a workspace: the library's fixed device scratch holds
@@ -203,16 +222,21 @@ def _hptr(t: Optional[torch.Tensor]):
     return t.data_ptr() or None
 
 
-def forward_args(*, q_idx, q_scale, w, k_idx, k_scale, q, kv, D_V, sm_scale, k, host=False):
+def forward_args(*, q_idx, q_scale, w, k_idx, k_scale, q, kv, D_V, sm_scale, k, host=False,
+                 kv_scale=None, kv_dtype=None):
     """The argument block of dsa_forward; host=True takes host tensors (the
-    `host` block of dsa_forward_host, where k_idx / k_scale / kv may be None)."""
+    `host` block of dsa_forward_host, where k_idx / k_scale / kv / kv_scale
+    may be None).  The MLA cache is bf16, or float8_e4m3fn codes with their
+    per-token kv_scale (kv_dtype is taken from kv, or given when kv is None)."""
     n_q, H_I, D_I = q_idx.shape
     _, H, D_K = q.shape
     f = _hptr if host else _ptr
+    if kv_dtype is None:
+        kv_dtype = DSA_E4M3 if kv is not None and kv.dtype == torch.float8_e4m3fn else DSA_BF16
     a = dsa_forward_args_t(_DTYPE_CODE[q_idx.dtype], H_I, D_I, f(q_idx), f(q_scale), f(w),
                            f(k_idx), f(k_scale), H, D_K, int(D_V), float(sm_scale), f(q),
-                           f(kv), int(k))
-    a._keep = (q_idx, q_scale, w, k_idx, k_scale, q, kv)
+                           f(kv), int(k), int(kv_dtype), f(kv_scale))
+    a._keep = (q_idx, q_scale, w, k_idx, k_scale, q, kv, kv_scale)
     return a
 
 

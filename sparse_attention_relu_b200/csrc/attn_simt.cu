@@ -23,10 +23,13 @@ constexpr int kHG = 16;       // heads per CTA
 constexpr int kChunk = 32;    // index slots per chunk
 constexpr int kThreads = 256;
 
-template <int VPT>  // output columns per thread: D_V <= 16 * VPT
+// FP8: the cache holds e4m3 codes with one fp32 scale per token (kv_scale);
+// a gathered row is decoded exactly and multiplied by its scale in fp32.
+template <int VPT, bool FP8>  // output columns per thread: D_V <= 16 * VPT
 __global__ void __launch_bounds__(kThreads) attn_simt_kernel(Rows R, int32_t row0,
                                                              const uint16_t* __restrict__ q,
-                                                             const uint16_t* __restrict__ kv,
+                                                             const void* __restrict__ kv,
+                                                             const float* __restrict__ kv_scale,
                                                              const int32_t* __restrict__ idx, int k,
                                                              int H, int D_K, int D_V, float sm_scale,
                                                              uint16_t* __restrict__ out,
@@ -58,7 +61,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(Rows R, int32_t row
 #pragma unroll
   for (int i = 0; i < VPT; ++i) acc[i] = 0.f;
 
-  const int nvec = D_K / 8;
+  const int nvec = FP8 ? D_K / 16 : D_K / 8;  // 16-byte vectors per cached row
   for (int c0 = 0; c0 < k; c0 += kChunk) {
     if (tid < kChunk) {
       int s = (c0 + tid < k) ? __ldg(irow + c0 + tid) : -1;
@@ -74,8 +77,29 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(Rows R, int32_t row
       int rr = i / nvec, vv = i - rr * nvec;
       int s = sel[rr];
       float* dst = cs + rr * (D_K + 1) + vv * 8;
-      if (s >= 0) {
-        uint4 v = __ldg(reinterpret_cast<const uint4*>(kv + (ri.kbase + s) * D_K) + vv);
+      if (FP8) {
+        float* d16 = cs + rr * (D_K + 1) + vv * 16;
+        if (s >= 0) {
+          const uint8_t* row = reinterpret_cast<const uint8_t*>(kv) + (ri.kbase + s) * D_K;
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(row) + vv);
+          const float sc = __ldg(kv_scale + ri.kbase + s);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint32_t lo, hi;
+            e4m3x4_to_bf16x4(w4[e], lo, hi);
+            d16[4 * e] = __uint_as_float(lo << 16) * sc;
+            d16[4 * e + 1] = __uint_as_float(lo & 0xffff0000u) * sc;
+            d16[4 * e + 2] = __uint_as_float(hi << 16) * sc;
+            d16[4 * e + 3] = __uint_as_float(hi & 0xffff0000u) * sc;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) d16[e] = 0.f;
+        }
+      } else if (s >= 0) {
+        const uint16_t* row = reinterpret_cast<const uint16_t*>(kv) + (ri.kbase + s) * D_K;
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(row) + vv);
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -152,32 +176,39 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(Rows R, int32_t row
 
 template <int VPT>
 dsa_status_t launch_v(const Rows& R, int32_t row0, int32_t nrows, const uint16_t* q,
-                      const uint16_t* kv, const int32_t* idx, int k, int H, int D_K, int D_V,
-                      float sm_scale, uint16_t* out, float* lse, cudaStream_t st) {
+                      const void* kv, const float* kv_scale, const int32_t* idx, int k, int H,
+                      int D_K, int D_V, float sm_scale, uint16_t* out, float* lse,
+                      cudaStream_t st) {
   size_t smem = sizeof(float) * ((size_t)kHG * D_K + (size_t)kChunk * (D_K + 1) +
                                  kHG * kChunk + 3 * kHG) +
                 sizeof(int) * kChunk;
-  auto kfn = attn_simt_kernel<VPT>;
+  auto kfn = kv_scale ? attn_simt_kernel<VPT, true> : attn_simt_kernel<VPT, false>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
   dim3 grid(nrows, (H + kHG - 1) / kHG);
-  kfn<<<grid, kThreads, smem, st>>>(R, row0, q, kv, idx, k, H, D_K, D_V, sm_scale, out, lse);
+  kfn<<<grid, kThreads, smem, st>>>(R, row0, q, kv, kv_scale, idx, k, H, D_K, D_V, sm_scale, out,
+                                    lse);
   return launch_status();
 }
 
 }  // namespace
 
 dsa_status_t launch_attn_simt(const Rows& R, int32_t row0, int32_t nrows, const uint16_t* q,
-                              const uint16_t* kv, const int32_t* idx, int k, int H, int D_K,
-                              int D_V, float sm_scale, uint16_t* out, float* lse, cudaStream_t st) {
+                              const void* kv, const float* kv_scale, const int32_t* idx, int k,
+                              int H, int D_K, int D_V, float sm_scale, uint16_t* out, float* lse,
+                              cudaStream_t st) {
   if (nrows <= 0) return DSA_OK;
+  if (kv_scale && D_K % 16) return DSA_ERR_UNSUPPORTED;  // 16-byte vectors of e4m3 codes
   const int vpt = (D_V + 15) / 16;
-  if (vpt <= 4) return launch_v<4>(R, row0, nrows, q, kv, idx, k, H, D_K, D_V, sm_scale, out, lse, st);
-  if (vpt <= 8) return launch_v<8>(R, row0, nrows, q, kv, idx, k, H, D_K, D_V, sm_scale, out, lse, st);
-  if (vpt <= 16) return launch_v<16>(R, row0, nrows, q, kv, idx, k, H, D_K, D_V, sm_scale, out, lse, st);
-  if (vpt <= 32) return launch_v<32>(R, row0, nrows, q, kv, idx, k, H, D_K, D_V, sm_scale, out, lse, st);
-  if (vpt <= 64) return launch_v<64>(R, row0, nrows, q, kv, idx, k, H, D_K, D_V, sm_scale, out, lse, st);
+#define DSA_LAUNCH_V(n) \
+  launch_v<n>(R, row0, nrows, q, kv, kv_scale, idx, k, H, D_K, D_V, sm_scale, out, lse, st)
+  if (vpt <= 4) return DSA_LAUNCH_V(4);
+  if (vpt <= 8) return DSA_LAUNCH_V(8);
+  if (vpt <= 16) return DSA_LAUNCH_V(16);
+  if (vpt <= 32) return DSA_LAUNCH_V(32);
+  if (vpt <= 64) return DSA_LAUNCH_V(64);
+#undef DSA_LAUNCH_V
   return DSA_ERR_UNSUPPORTED;
 }
 

@@ -79,6 +79,9 @@ constexpr int kAtomsA = 5, kAtomsV = 4;
 constexpr int kChunksA = kNT * kAtomsA * 8;    // 2560 16-byte chunks
 constexpr int kChunksV = kNT * kAtomsV * 8;    // 2048
 constexpr int kIdxRing = 4;                    // tiles whose indices are held
+// e4m3 cache: a 16-byte load brings 16 codes, two 16-byte bf16 chunks of the
+// swizzled operand, so each group takes half as many loads as chunks.
+constexpr int kLoadsA = kChunksA / 2, kLoadsV = kChunksV / 2;  // 1280, 1024
 constexpr int kQTmemDims = 384;                // query dims held in TMEM
 constexpr int kQSmemAtoms = (kDK - kQTmemDims) / 64;  // 3 atoms in shared memory
 constexpr int kQAtomBytes = kH * 128;          // 16384
@@ -89,8 +92,9 @@ constexpr int OFF_P = OFF_Q + kQSmemAtoms * kQAtomBytes;
 constexpr int OFF_IDX = OFF_P + kPBytes;                 // [ring][64] int32
 constexpr int OFF_MASK = OFF_IDX + kIdxRing * kNT * 4;   // [ring][2] uint32 validity bits
 constexpr int OFF_HMAX = OFF_MASK + kIdxRing * 2 * 4;    // [2 tiles][2 warpgroups][128] float
-constexpr int OFF_BAR = OFF_HMAX + 2 * 2 * kH * 4;
-constexpr int kNumBars = 16;
+constexpr int OFF_KSC = OFF_HMAX + 2 * 2 * kH * 4;       // [ring][64] fp32 cache scales (e4m3)
+constexpr int OFF_BAR = OFF_KSC + kIdxRing * kNT * 4;
+constexpr int kNumBars = 18;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 // The dynamic window starts 1024-aligned (right after the driver's reserved
 // kilobyte, with no static shared memory); the kernel checks it.
@@ -102,7 +106,11 @@ constexpr uint32_t TM_Q = 0;     // query dims 0..383 of all heads, bf16 pairs (
 constexpr uint32_t TM_S = 192;   // 64-column score tile
 constexpr uint32_t TM_O = 256;   // 256-column output accumulator
 constexpr uint32_t IDESC_QK = idesc(1, 128, kNT);
-constexpr uint32_t IDESC_PV = idesc(1, 128, 256, false, true);
+// PV runs as N = 64 MMAs (one per 64 value columns): the QK MMAs are N = 64,
+// and a stream that mixes MMA shapes was measured on B200 to take about twice
+// the time of its parts.
+constexpr int kPvN = 64;
+constexpr uint32_t IDESC_PV = idesc(1, 128, kPvN, false, true);
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;  // log2 headroom before the reference max moves
@@ -118,9 +126,9 @@ enum {
   B_PFULL = 11,   // P stored (every softmax thread)
   B_PVDONE = 12,  // PV retired
   B_DRAIN = 13,
-  B_IDX = 14      // [2] the tile's indices are in the ring (producers)
+  B_IDX = 14      // [kIdxRing] the tile's indices, mask and scales are in the ring (producers)
 };
-static_assert(B_DRAIN < kNumBars, "barrier count");
+static_assert(B_IDX + kIdxRing <= kNumBars, "barrier count");
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
@@ -187,6 +195,27 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// 16 bytes of read-only global memory, not kept in L1.
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// 16 e4m3 codes (dims 16c .. 16c+15 of a 64-dim atom row) -> the two 16-byte
+// bf16 chunks 2c, 2c+1 of that row at `rowp`, in the 128-byte swizzle.
+__device__ __forceinline__ void store_codes(uint8_t* rowp, int c, int row, const uint4& x) {
+  uint4 a, b;
+  e4m3x4_to_bf16x4(x.x, a.x, a.y);
+  e4m3x4_to_bf16x4(x.y, a.z, a.w);
+  e4m3x4_to_bf16x4(x.z, b.x, b.y);
+  e4m3x4_to_bf16x4(x.w, b.z, b.w);
+  *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (row & 7)) << 4)) = a;
+  *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (row & 7)) << 4)) = b;
+}
+
 struct Split {
   int nsplit, tiles_per_split;
 };
@@ -224,8 +253,15 @@ inline Split plan_split(int32_t nrows, int k) {
   return best;
 }
 
+// FP8: the cache holds e4m3 codes [n_k, 576] with one fp32 scale per token
+// (kv_scale).  The codes are gathered through registers and written to the
+// same swizzled bf16 operand, exactly converted; the MMAs are the bf16 ones.
+// The token's scale multiplies its score column and its probability in the
+// PV operand (P' = p * scale); the softmax denominator sums p.
+template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kv, Rows R,
+    attn_tc_kernel(const uint16_t* __restrict__ q, const void* __restrict__ kv,
+                   const float* __restrict__ kv_scale, Rows R,
                    int32_t row0, const int32_t* __restrict__ idx, int k, float scale2, Split sp,
                    uint16_t* __restrict__ out, float* __restrict__ lse,
                    float* __restrict__ part_o, float* __restrict__ part_lse) {
@@ -239,7 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t* sidx = reinterpret_cast<int32_t*>(smem + OFF_IDX);
   uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + OFF_MASK);
   float* hmax = reinterpret_cast<float*>(smem + OFF_HMAX);
+  float* ksc = reinterpret_cast<float*>(smem + OFF_KSC);
   auto bar = [&](int i) { return sb + OFF_BAR + 8u * i; };
+  constexpr int kRowBytes = FP8 ? kDK : kDK * 2;  // one cached token
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -258,12 +296,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kStages; ++i) {
       // per producer: an arrive after the index store and a cp.async arrive
       mbar_init(bar(B_AFULL + i), 2 * kProducers);
-      mbar_init(bar(B_VFULL + i), kSoftmaxThreads);  // a cp.async arrive per softmax thread
-      mbar_init(bar(B_IDX + i), kProducers);
+      mbar_init(bar(B_VFULL + i), kProducers);  // a cp.async arrive (or arrive) per producer
       mbar_init(bar(B_AEMPTY + i), 1);
       mbar_init(bar(B_VEMPTY + i), 1);
     }
     mbar_init(bar(B_SFULL), 1);
+    for (int i = 0; i < kIdxRing; ++i) mbar_init(bar(B_IDX + i), kProducers);
     mbar_init(bar(B_SEMPTY), kSoftmaxThreads);
     mbar_init(bar(B_PFULL), kSoftmaxThreads);
     mbar_init(bar(B_PVDONE), 1);
@@ -280,41 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Group V of tile n (this CTA's value columns, 2048 16-byte chunks) is
-  // fetched by the softmax threads, which are otherwise idle while the
-  // tensor cores work on the next tile; thread t issues chunks t + 256 j.
-  // Indices come from the ring the producers fill.
-  const char* const kvrow0 = reinterpret_cast<const char*>(kv + ri.kbase * kDK);
-  auto issue_v = [&](int n) {
-    const int st = n % kStages, ring = n % kIdxRing, t = tid - kSoftmax0;
-#pragma unroll
-    for (int j = 0; j < kChunksV / kSoftmaxThreads; ++j) {
-      const int i = t + kSoftmaxThreads * j;
-      const int ch = i & 7, seg = i >> 3, row = seg >> 2, atom = 4 * half + (seg & 3);
-      const int32_t s = sidx[ring * kNT + row];
-      const char* src = s >= 0 ? kvrow0 + (int64_t)s * (kDK * 2) + atom * 128 + ch * 16
-                               : reinterpret_cast<const char*>(kv);
-      const uint32_t nbytes = s >= 0 ? 16u : 0u;  // 0: zero-fill
-      const uint32_t dst = sb + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128 +
-                           ((uint32_t)(ch ^ (row & 7)) << 4);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                   "r"(nbytes)
-                   : "memory");
-    }
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_VFULL + st))
-                 : "memory");
-  };
-  // Waits until group V of tile n may be fetched: its indices are published
-  // and PV(n-2) released the stage's value atoms.
-  auto v_ready = [&](int n) -> bool {
-    const int st = n % kStages;
-    return mbar_wait(bar(B_IDX + st), (n / kStages) & 1, R.status) &&
-           mbar_wait(bar(B_VEMPTY + st), ((n / kStages) & 1) ^ 1, R.status);
-  };
-
   if (warp < kMmaWarp) {
     // ------------------------------------------------------------ gather producer
-    const char* kvb = reinterpret_cast<const char*>(kv + ri.kbase * kDK);
+    const char* kvb = reinterpret_cast<const char*>(kv) + ri.kbase * kRowBytes;
     auto load_idx = [&](int n) -> int32_t {
       const int slot = slot_lo + n * kNT + tid;
       int32_t s = slot < slot_hi ? __ldg(idx + (int64_t)rloc * k + slot) : -1;
@@ -325,8 +331,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return s;
     };
-    // Threads 0..63 own the index of tile row tid.
+    // the scale of cache row s of this sequence (e4m3 cache), 0 for an empty slot
+    auto load_scale = [&](int32_t s) -> float {
+      return (FP8 && s >= 0) ? __ldg(kv_scale + ri.kbase + s) : 0.f;
+    };
+    // Threads 0..63 own the index (and scale) of tile row tid.
     int32_t pre = (tid < kNT && ntiles > 0) ? load_idx(0) : -1;
+    float pre_sc = load_scale(pre);
     // Issues 16-byte chunk i of group G (eight lanes per 128-byte segment of
     // a row, a warp four consecutive segments) of tile n into stage st.
     auto issue = [&](int st, int ring, int i, bool group_a) {
@@ -341,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         atom = 4 * half + (seg & 3);
       }
       const int32_t s = sidx[ring * kNT + row];
-      const char* src = s >= 0 ? kvb + (int64_t)s * (kDK * 2) + atom * 128 + ch * 16
+      const char* src = s >= 0 ? kvb + (int64_t)s * kRowBytes + atom * 128 + ch * 16
                                : reinterpret_cast<const char*>(kv);
       const uint32_t nbytes = s >= 0 ? 16u : 0u;  // 0: zero-fill
       const uint32_t dst = sb + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128 +
@@ -361,18 +372,83 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (tid < kNT) {
         sidx[ring * kNT + tid] = pre;
+        if (FP8) ksc[ring * kNT + tid] = pre_sc;
         const uint32_t bits = __ballot_sync(0xffffffffu, pre >= 0);
         if (lane == 0) vmask[ring * 2 + warp] = bits;
       }
-      mbar_arrive(bar(B_AFULL + st));  // publishes indices and mask to the softmax threads
-      mbar_arrive(bar(B_IDX + st));    // ... and to the threads fetching group V
+      mbar_arrive(bar(B_AFULL + st));   // publishes indices to the MMA issuer
+      mbar_arrive(bar(B_IDX + ring));   // ... and indices, mask, scales to the softmax threads
       asm volatile("bar.sync 2, %0;" ::"n"(kProducers) : "memory");  // producers see the indices
-      if (tid < kNT) pre = n + 1 < ntiles ? load_idx(n + 1) : -1;  // overlaps the copies below
+      if (tid < kNT) {  // overlaps the copies below
+        pre = n + 1 < ntiles ? load_idx(n + 1) : -1;
+        pre_sc = load_scale(pre);
+      }
+      if constexpr (FP8) {
+        // group A through registers: all loads in flight, then convert and store
+        constexpr int J = (kLoadsA + kProducers - 1) / kProducers;
+        uint4 x[J];
 #pragma unroll
-      for (int j = 0; j < (kChunksA + kProducers - 1) / kProducers; ++j)
-        if (tid + kProducers * j < kChunksA) issue(st, ring, tid + kProducers * j, true);
-      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar(B_AFULL + st))
-                   : "memory");
+        for (int j = 0; j < J; ++j) {
+          const int i = tid + kProducers * j, c = i & 3, seg = i >> 2, row = seg / kAtomsA;
+          const int ai = seg - row * kAtomsA, atom = ai < 4 ? 4 * (half ^ 1) + ai : 8;
+          const int32_t s = i < kLoadsA ? sidx[ring * kNT + row] : -1;
+          x[j] = s >= 0 ? ld_nc_v4(kvb + (int64_t)s * kRowBytes + atom * 64 + c * 16)
+                        : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+          const int i = tid + kProducers * j, c = i & 3, seg = i >> 2, row = seg / kAtomsA;
+          const int ai = seg - row * kAtomsA, atom = ai < 4 ? 4 * (half ^ 1) + ai : 8;
+          if (i < kLoadsA)
+            store_codes(smem + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128, c, row, x[j]);
+        }
+        fence_async_smem();
+        mbar_arrive(bar(B_AFULL + st));
+      } else {
+#pragma unroll
+        for (int j = 0; j < (kChunksA + kProducers - 1) / kProducers; ++j)
+          if (tid + kProducers * j < kChunksA) issue(st, ring, tid + kProducers * j, true);
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
+                         bar(B_AFULL + st))
+                     : "memory");
+      }
+      // group V of the stage (this CTA's value columns) is free once PV(n-2)
+      // read it; the producers fetch it too, so that the softmax threads never
+      // wait for a PV to retire
+      ok = mbar_wait(bar(B_VEMPTY + st), par, R.status) && !*abort_flag;
+      if (!bar_and<2, kProducers>(ok)) {
+        *abort_flag = 1;
+        break;
+      }
+      if constexpr (FP8) {
+        // 16 codes per load: segment (row, atom) quarter c holds dims 16c .. 16c+15
+        constexpr int J = (kLoadsV + kProducers - 1) / kProducers;
+        uint4 x[J];
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+          const int i = tid + kProducers * j, c = i & 3, seg = i >> 2, row = seg >> 2;
+          const int atom = 4 * half + (seg & 3);
+          const int32_t s = i < kLoadsV ? sidx[ring * kNT + row] : -1;
+          x[j] = s >= 0 ? ld_nc_v4(kvb + (int64_t)s * kRowBytes + atom * 64 + c * 16)
+                        : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+          const int i = tid + kProducers * j, c = i & 3, seg = i >> 2, row = seg >> 2;
+          const int atom = 4 * half + (seg & 3);
+          if (i < kLoadsV)
+            store_codes(smem + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128, c, row, x[j]);
+        }
+        fence_async_smem();
+        mbar_arrive(bar(B_VFULL + st));
+      } else {
+#pragma unroll
+        for (int j = 0; j < (kChunksV + kProducers - 1) / kProducers; ++j)
+          if (tid + kProducers * j < kChunksV) issue(st, ring, tid + kProducers * j, false);
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
+                         bar(B_VFULL + st))
+                     : "memory");
+      }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kMmaWarp) {
@@ -420,8 +496,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               sb + OFF_C + (np % kStages) * kCBytes + 4 * half * kAtomBytes, kAtomBytes, 1024);
 #pragma unroll
           for (int kk = 0; kk < kNT / 16; ++kk)
-            mma_bf16(tmem + TM_O, dp0 + (uint64_t)(kk * 2), dv + (uint64_t)(kk * 128), IDESC_PV,
-                     (np > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int a = 0; a < 256 / kPvN; ++a)  // 64-column blocks are atoms kAtomBytes apart
+              mma_bf16(tmem + TM_O + kPvN * a, dp0 + (uint64_t)(kk * 2),
+                       dv + (uint64_t)(kk * 128 + a * (kPvN / 64) * (kAtomBytes >> 4)), IDESC_PV,
+                       (np > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(B_PVDONE));
           mma_commit(bar(B_VEMPTY + np % kStages));
           ++np;
@@ -529,13 +608,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_QREADY));
     }
-    // group V of the first two tiles
-    for (int n = 0; n < kStages && n < ntiles; ++n) {
-      if (v_ready(n))
-        issue_v(n);
-      else
-        *abort_flag = 1;
-    }
     // row h of P: this warpgroup's 32 rows are 16-byte chunks 4wg .. 4wg+3
     uint8_t* const prow = smem + OFF_P + h * 128;
     float m2 = -INFINITY, l = 0.f;
@@ -543,12 +615,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int n = 0; ok && n < ntiles; ++n) {
       const int st = n % kStages;
       float s[32];
-      // S(n) retired.  The tile's validity bits are already visible: this
-      // thread waited for their publication (B_IDX) before fetching the
-      // tile's group V.  (No wait on B_AFULL here: the producers may already
-      // have refilled the stage's group A for tile n+2, two phases on, which
-      // a parity wait would never see complete.)
-      bool w_ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), n & 1, R.status) && !*abort_flag);
+      // S(n) retired; then the tile's validity bits and scales are visible
+      // (B_IDX: the producers published them; they cannot publish tile n+4
+      // into this slot before this thread has read S(n+1), so the parity
+      // names tile n's phase)
+      bool w_ok = __all_sync(0xffffffffu,
+                             mbar_wait(bar(B_SFULL), n & 1, R.status) &&
+                                 mbar_wait(bar(B_IDX + n % kIdxRing), (n / kIdxRing) & 1,
+                                           R.status) &&
+                                 !*abort_flag);
       if (w_ok) {
         tc_fence_after();
         tmem_ld32(tmem + lane_off + TM_S + 32 * wg, s);
@@ -559,10 +634,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const uint32_t bits = vmask[(n % kIdxRing) * 2 + wg];
       mbar_arrive(bar(B_SEMPTY));  // the MMA may overwrite the score tile
+      // this warpgroup's 32 rows of the tile: their cache scales (e4m3); the
+      // ring entry stays until the producers refill it four tiles on
+      const float* const tsc = ksc + (n % kIdxRing) * kNT + 32 * wg;
       float hm = -INFINITY;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        s[j] = ((bits >> j) & 1u) ? s[j] * scale2 : -INFINITY;
+        const float sc = FP8 ? scale2 * tsc[j] : scale2;
+        s[j] = ((bits >> j) & 1u) ? s[j] * sc : -INFINITY;
         hm = fmaxf(hm, s[j]);
       }
       float* const hm_buf = hmax + (n & 1) * (2 * kH);  // two tiles in flight
@@ -599,8 +678,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < 16; ++j) {
         const float p0 = ex2(s[2 * j] - mref);
         const float p1 = ex2(s[2 * j + 1] - mref);
-        pw[j] = pack_bf16(p0, p1);  // bf16 only as the MMA operand
-        lsum += p0 + p1;            // the denominator keeps fp32 probabilities
+        if (FP8)  // the PV operand carries each token's cache scale: P' = p * scale
+          pw[j] = pack_bf16(p0 * tsc[2 * j], p1 * tsc[2 * j + 1]);
+        else
+          pw[j] = pack_bf16(p0, p1);  // bf16 only as the MMA operand
+        lsum += p0 + p1;              // the denominator keeps fp32 probabilities
       }
       if (t_ok) {
 #pragma unroll
@@ -613,16 +695,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();          // P stores before the PV MMA reads them
       tc_fence_before();           // a rescale's TMEM stores before the PV MMA
       mbar_arrive(bar(B_PFULL));
-      // group V of tile n+2 goes into this stage once PV(n) has read it
-      if (n + kStages < ntiles) {
-        if (v_ready(n + kStages))
-          issue_v(n + kStages);
-        else
-          *abort_flag = 1;
-      }
     }
     if (!ok) *abort_flag = 1;
-    asm volatile("cp.async.wait_all;" ::: "memory");  // no group-V copy outlives the CTA
     // combine the two warpgroups' denominators (the first barrier retires the
     // last tile's reads of the half maxima)
     asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -729,8 +803,8 @@ size_t attn_tc_workspace(int32_t nrows, int k, int H, int D_V) {
 }
 
 dsa_status_t launch_attn_tc(const Rows& R, int32_t row0, int32_t nrows, const uint16_t* q,
-                            const uint16_t* kv, const int32_t* idx, int k, float sm_scale,
-                            uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                            const void* kv, const float* kv_scale, const int32_t* idx, int k,
+                            float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
                             cudaStream_t st) {
   if (nrows <= 0) return DSA_OK;
   const Split sp = plan_split(nrows, k);
@@ -740,12 +814,12 @@ dsa_status_t launch_attn_tc(const Rows& R, int32_t row0, int32_t nrows, const ui
     part_o = reinterpret_cast<float*>(ws);
     part_lse = part_o + (size_t)nrows * sp.nsplit * kH * kDV;
   }
-  if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
-      cudaSuccess)
+  auto kfn = kv_scale ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
     return DSA_ERR_CUDA;
   const dim3 grid(2 * nrows * sp.nsplit);
-  attn_tc_kernel<<<grid, kThreads, kSmem, st>>>(q, kv, R, row0, idx, k, sm_scale * kLog2e, sp,
-                                                out, lse, part_o, part_lse);
+  kfn<<<grid, kThreads, kSmem, st>>>(q, kv, kv_scale, R, row0, idx, k, sm_scale * kLog2e, sp, out,
+                                     lse, part_o, part_lse);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (sp.nsplit > 1) {
     attn_combine_kernel<<<dim3(nrows, kH), 128, 0, st>>>(row0, sp.nsplit, part_o, part_lse, out,
@@ -780,7 +854,8 @@ dsa_status_t launch_attn_tc_static(const Rows& R, int32_t row0, int32_t nrows, c
     }
     scratch = addr[dev];
   }
-  return launch_attn_tc(R, row0, nrows, q, kv, idx, k, sm_scale, out, lse, scratch, need, st);
+  return launch_attn_tc(R, row0, nrows, q, kv, nullptr, idx, k, sm_scale, out, lse, scratch, need,
+                        st);
 }
 
 }  // namespace dsa

@@ -101,6 +101,23 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
 }
 
+// Four e4m3 codes (c0 in the low byte of w) -> bf16 pairs {c0, c1}, {c2, c3},
+// exactly: each code's exponent and mantissa bits move into a bf16 with the
+// exponent bias of e4m3's unbiased field (a bf16 subnormal when the code is
+// subnormal), and one exact multiplication by 2^120 rebiases 7 -> 127 for
+// normal and subnormal codes alike.  (The NaN codes S.1111.111 come out as
+// +-480; the cache holds none.)
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  uint32_t a, b;
+  asm("prmt.b32 %0, %1, 0, 0x4140;" : "=r"(a) : "r"(w));  // c0, c1 in the low bytes of halves
+  asm("prmt.b32 %0, %1, 0, 0x4342;" : "=r"(b) : "r"(w));  // c2, c3
+  a = ((a << 4) & 0x07F007F0u) | ((a << 8) & 0x80008000u);
+  b = ((b << 4) & 0x07F007F0u) | ((b << 8) & 0x80008000u);
+  const uint32_t k2p120 = 0x7B807B80u;  // bf16x2 {2^120, 2^120}
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(k2p120));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(k2p120));
+}
+
 // Host-side launch error helper.
 inline dsa_status_t launch_status() {
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;

@@ -102,11 +102,18 @@ dsa_status_t check_indexer(const Rows& R, const void* q_idx, const float* q_scal
   return DSA_OK;
 }
 
-dsa_status_t check_attn(const Rows& R, const void* q, const void* kv, int k, int H, int D_K,
-                        int D_V, float sm_scale, const void* out, const float* lse) {
+// kv_dtype: DSA_BF16, or DSA_E4M3 with kv_scale [n_k] (the per-token scales).
+dsa_status_t check_attn(const Rows& R, const void* q, const void* kv, int kv_dtype,
+                        const float* kv_scale, int k, int H, int D_K, int D_V, float sm_scale,
+                        const void* out, const float* lse) {
   if (k < 1 || k > 16384) return DSA_ERR_INVALID_ARGUMENT;
   if (H < 1 || H > 128 || D_K < 8 || D_K > 1024 || D_K % 8 || D_V < 8 || D_V > D_K || D_V % 8)
     return DSA_ERR_INVALID_ARGUMENT;
+  if (kv_dtype == DSA_E4M3) {
+    if (D_K % 16 || !ptr_ok(kv_scale, R.n_k > 0)) return DSA_ERR_INVALID_ARGUMENT;
+  } else if (kv_dtype != DSA_BF16 || kv_scale) {
+    return DSA_ERR_INVALID_ARGUMENT;
+  }
   if (!isfinite(sm_scale)) return DSA_ERR_INVALID_ARGUMENT;
   const bool rows = R.n_q > 0;
   if (!ptr_ok(q, rows) || !ptr_ok(kv, R.n_k > 0) || !ptr_ok(out, rows))
@@ -130,14 +137,16 @@ size_t attn_ws(int32_t nrows, int k, int H, int D_K, int D_V) {
   return attn_tc_supported(H, D_K, D_V) ? attn_tc_workspace(nrows, k, H, D_V) : 0;
 }
 
+// kv_scale != NULL: an e4m3 cache with per-token scales, else bf16.
 dsa_status_t run_attn(const Rows& R, int32_t row0, int32_t nrows, const void* q, const void* kv,
-                      const int32_t* idx, int k, int H, int D_K, int D_V, float sm_scale,
-                      void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
+                      const float* kv_scale, const int32_t* idx, int k, int H, int D_K, int D_V,
+                      float sm_scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                      cudaStream_t st) {
   if (attn_tc_supported(H, D_K, D_V))
-    return launch_attn_tc(R, row0, nrows, (const uint16_t*)q, (const uint16_t*)kv, idx, k,
-                          sm_scale, (uint16_t*)out, lse, ws, ws_bytes, st);
-  return launch_attn_simt(R, row0, nrows, (const uint16_t*)q, (const uint16_t*)kv, idx, k, H, D_K,
-                          D_V, sm_scale, (uint16_t*)out, lse, st);
+    return launch_attn_tc(R, row0, nrows, (const uint16_t*)q, kv, kv_scale, idx, k, sm_scale,
+                          (uint16_t*)out, lse, ws, ws_bytes, st);
+  return launch_attn_simt(R, row0, nrows, (const uint16_t*)q, kv, kv_scale, idx, k, H, D_K, D_V,
+                          sm_scale, (uint16_t*)out, lse, st);
 }
 
 constexpr size_t kAlign = 256;
@@ -155,20 +164,29 @@ int32_t slab_rows(const Rows& R) {
   return (int32_t)rows;
 }
 
+// The fused decode selection is built and tested but not yet faster than the
+// separate top-k kernel, so dsa_forward does not take it.
+constexpr bool kFusedDecodeSelect = false;
+
 struct ForwardPlan {
   int32_t slab;
+  bool fused;  // decode: indexer and top-k in one kernel, no score rows
   size_t off_scores, off_idx, off_attn, total;
 };
 
-// slab_cap > 0 caps the rows per slab below the scores bound.
+// slab_cap > 0 caps the rows per slab below the scores bound.  Decode rows
+// (tensor-core indexer) take the fused indexer + selection: the workspace then
+// holds the rows' candidate lists instead of their scores.
 ForwardPlan plan_forward(const Rows& R, const dsa_forward_args_t* a, bool own_idx,
                          int32_t slab_cap = 0) {
   ForwardPlan p{};
   p.slab = slab_rows(R);
   if (slab_cap > 0 && slab_cap < p.slab) p.slab = slab_cap;
+  p.fused = kFusedDecodeSelect && indexer_select_supported(R, a->idx_dtype, a->H_I, a->D_I, a->k);
   size_t o = 0;
   p.off_scores = o;
-  o = align_up(o + (size_t)p.slab * R.max_len * 4);
+  o = align_up(o + (p.fused ? indexer_select_workspace(R, p.slab)
+                            : (size_t)p.slab * R.max_len * 4));
   p.off_idx = o;
   if (own_idx) o = align_up(o + (size_t)p.slab * a->k * 4);
   p.off_attn = o;
@@ -201,8 +219,10 @@ dsa_status_t copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
 dsa_status_t check_host(const Rows& R, const dsa_forward_args_t* h, const dsa_forward_args_t* d,
                         const void* host_out, const float* host_lse, const float* dev_lse) {
   if (h->idx_dtype != d->idx_dtype || h->H_I != d->H_I || h->D_I != d->D_I || h->H != d->H ||
-      h->D_K != d->D_K || h->D_V != d->D_V || h->k != d->k || !(h->sm_scale == d->sm_scale))
+      h->D_K != d->D_K || h->D_V != d->D_V || h->k != d->k || !(h->sm_scale == d->sm_scale) ||
+      h->kv_dtype != d->kv_dtype)
     return DSA_ERR_INVALID_ARGUMENT;
+  if (d->kv_dtype != DSA_E4M3 && h->kv_scale) return DSA_ERR_INVALID_ARGUMENT;
   const bool rows = R.n_q > 0, e4m3 = d->idx_dtype == DSA_E4M3;
   if (rows && (!h->q_idx || !h->w || !h->q || !host_out || (e4m3 && !h->q_scale)))
     return DSA_ERR_INVALID_ARGUMENT;
@@ -227,6 +247,24 @@ struct CallEvents {
   }
 };
 
+dsa_status_t sparse_mla_attn(const dsa_layout_t* layout, const void* q, const void* kv,
+                             int kv_dtype, const float* kv_scale, const int32_t* idx, int32_t k,
+                             int32_t H, int32_t D_K, int32_t D_V, float sm_scale, void* out,
+                             float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  Rows R;
+  dsa_status_t s = check_layout(layout, &R);
+  if (s) return s;
+  if ((s = check_attn(R, q, kv, kv_dtype, kv_scale, k, H, D_K, D_V, sm_scale, out, lse)))
+    return s;
+  if (!ptr_ok(idx, R.n_q > 0)) return DSA_ERR_INVALID_ARGUMENT;
+  const size_t need = attn_ws(R.n_q, k, H, D_K, D_V);
+  if (need && (!workspace || ws_bytes < need || !aligned16(workspace))) return DSA_ERR_WORKSPACE;
+  if (R.n_q == 0) return DSA_OK;
+  if ((s = device_rows(&R))) return s;
+  return run_attn(R, 0, R.n_q, q, kv, kv_scale, idx, k, H, D_K, D_V, sm_scale, out, lse,
+                  workspace, ws_bytes, (cudaStream_t)stream);
+}
+
 }  // namespace
 }  // namespace dsa
 
@@ -234,7 +272,7 @@ using namespace dsa;
 
 extern "C" {
 
-int32_t dsa_abi_version(void) { return 3; }
+int32_t dsa_abi_version(void) { return 4; }
 
 const char* dsa_status_string(dsa_status_t s) {
   switch (s) {
@@ -307,21 +345,22 @@ size_t dsa_sparse_mla_attn_workspace_size(const dsa_layout_t* layout, int32_t k,
   return attn_ws(R.n_q, k, H, D_K, D_V);
 }
 
+
 dsa_status_t dsa_sparse_mla_attn(const dsa_layout_t* layout, const void* q, const void* kv,
                                  const int32_t* idx, int32_t k, int32_t H, int32_t D_K,
                                  int32_t D_V, float sm_scale, void* out, float* lse,
                                  void* workspace, size_t ws_bytes, void* stream) {
-  Rows R;
-  dsa_status_t s = check_layout(layout, &R);
-  if (s) return s;
-  if ((s = check_attn(R, q, kv, k, H, D_K, D_V, sm_scale, out, lse))) return s;
-  if (!ptr_ok(idx, R.n_q > 0)) return DSA_ERR_INVALID_ARGUMENT;
-  const size_t need = attn_ws(R.n_q, k, H, D_K, D_V);
-  if (need && (!workspace || ws_bytes < need || !aligned16(workspace))) return DSA_ERR_WORKSPACE;
-  if (R.n_q == 0) return DSA_OK;
-  if ((s = device_rows(&R))) return s;
-  return run_attn(R, 0, R.n_q, q, kv, idx, k, H, D_K, D_V, sm_scale, out, lse, workspace,
-                  ws_bytes, (cudaStream_t)stream);
+  return sparse_mla_attn(layout, q, kv, DSA_BF16, nullptr, idx, k, H, D_K, D_V, sm_scale, out, lse,
+                         workspace, ws_bytes, stream);
+}
+
+dsa_status_t dsa_sparse_mla_attn_e4m3(const dsa_layout_t* layout, const void* q, const void* kv,
+                                      const float* kv_scale, const int32_t* idx, int32_t k,
+                                      int32_t H, int32_t D_K, int32_t D_V, float sm_scale,
+                                      void* out, float* lse, void* workspace, size_t ws_bytes,
+                                      void* stream) {
+  return sparse_mla_attn(layout, q, kv, DSA_E4M3, kv_scale, idx, k, H, D_K, D_V, sm_scale, out,
+                         lse, workspace, ws_bytes, stream);
 }
 
 dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_layout_t* layout, const void* q,
@@ -331,7 +370,7 @@ dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_layout_t* layout, const void*
   Rows R;
   dsa_status_t s = check_layout(layout, &R);
   if (s) return s;
-  if ((s = check_attn(R, q, kv, k, H, D_K, D_V, sm_scale, out, lse))) return s;
+  if ((s = check_attn(R, q, kv, DSA_BF16, nullptr, k, H, D_K, D_V, sm_scale, out, lse))) return s;
   if (!ptr_ok(idx, R.n_q > 0)) return DSA_ERR_INVALID_ARGUMENT;
   if (attn_tc_supported(H, D_K, D_V) &&
       attn_tc_workspace(R.n_q, k, H, D_V) > attn_tc_static_scratch_bytes())
@@ -341,8 +380,8 @@ dsa_status_t dsa_sparse_mla_attn_noalloc(const dsa_layout_t* layout, const void*
   if (attn_tc_supported(H, D_K, D_V))
     return launch_attn_tc_static(R, 0, R.n_q, (const uint16_t*)q, (const uint16_t*)kv, idx, k,
                                  sm_scale, (uint16_t*)out, lse, (cudaStream_t)stream);
-  return launch_attn_simt(R, 0, R.n_q, (const uint16_t*)q, (const uint16_t*)kv, idx, k, H, D_K,
-                          D_V, sm_scale, (uint16_t*)out, lse, (cudaStream_t)stream);
+  return launch_attn_simt(R, 0, R.n_q, (const uint16_t*)q, kv, nullptr, idx, k, H, D_K, D_V,
+                          sm_scale, (uint16_t*)out, lse, (cudaStream_t)stream);
 }
 
 size_t dsa_forward_workspace_size(const dsa_layout_t* layout, const dsa_forward_args_t* a) {
@@ -362,7 +401,8 @@ dsa_status_t dsa_forward_timed(const dsa_layout_t* layout, const dsa_forward_arg
   if ((s = check_indexer(R, a->q_idx, a->q_scale, a->w, a->k_idx, a->k_scale, a->idx_dtype,
                          a->H_I, a->D_I)))
     return s;
-  if ((s = check_attn(R, a->q, a->kv, a->k, a->H, a->D_K, a->D_V, a->sm_scale, out, lse)))
+  if ((s = check_attn(R, a->q, a->kv, a->kv_dtype, a->kv_scale, a->k, a->H, a->D_K, a->D_V,
+                      a->sm_scale, out, lse)))
     return s;
   if (idx_out && !aligned16(idx_out)) return DSA_ERR_INVALID_ARGUMENT;
   if (n_events > 0 && !events) return DSA_ERR_INVALID_ARGUMENT;
@@ -389,13 +429,22 @@ dsa_status_t dsa_forward_timed(const dsa_layout_t* layout, const dsa_forward_arg
   for (int32_t r0 = 0; r0 < R.n_q; r0 += p.slab) {
     const int32_t nr = (R.n_q - r0) < p.slab ? (R.n_q - r0) : p.slab;
     int32_t* idx = idx_out ? idx_out + (int64_t)r0 * a->k : (int32_t*)(ws + p.off_idx);
-    if ((s = run_indexer(R, r0, nr, a->idx_dtype, a->H_I, a->D_I, a->q_idx, a->q_scale, a->w,
-                         a->k_idx, a->k_scale, scores, false, st)))
-      return s;
-    if ((s = mark(0))) return s;
-    if ((s = launch_topk(R, r0, nr, scores, R.max_len, a->k, idx, st))) return s;
-    if ((s = mark(1))) return s;
-    if ((s = run_attn(R, r0, nr, a->q, a->kv, idx, a->k, a->H, a->D_K, a->D_V, a->sm_scale, out,
+    if (p.fused) {  // indexer and top-k in one kernel
+      if ((s = launch_indexer_select(R, r0, nr, a->idx_dtype, a->H_I, a->D_I, a->q_idx,
+                                     a->q_scale, a->w, a->k_idx, a->k_scale, a->k, idx, scores,
+                                     p.off_idx - p.off_scores, st)))
+        return s;
+      if ((s = mark(0))) return s;
+    } else {
+      if ((s = run_indexer(R, r0, nr, a->idx_dtype, a->H_I, a->D_I, a->q_idx, a->q_scale, a->w,
+                           a->k_idx, a->k_scale, scores, false, st)))
+        return s;
+      if ((s = mark(0))) return s;
+      if ((s = launch_topk(R, r0, nr, scores, R.max_len, a->k, idx, st))) return s;
+      if ((s = mark(1))) return s;
+    }
+    if ((s = run_attn(R, r0, nr, a->q, a->kv, a->kv_scale, idx, a->k, a->H, a->D_K, a->D_V,
+                      a->sm_scale, out,
                       lse, ws + p.off_attn, p.total - p.off_attn, st)))
       return s;
     if ((s = mark(2))) return s;
@@ -429,7 +478,8 @@ dsa_status_t dsa_forward_host(const dsa_layout_t* layout, const dsa_forward_args
   if ((s = check_indexer(R, a->q_idx, a->q_scale, a->w, a->k_idx, a->k_scale, a->idx_dtype,
                          a->H_I, a->D_I)))
     return s;
-  if ((s = check_attn(R, a->q, a->kv, a->k, a->H, a->D_K, a->D_V, a->sm_scale, dev_out,
+  if ((s = check_attn(R, a->q, a->kv, a->kv_dtype, a->kv_scale, a->k, a->H, a->D_K, a->D_V,
+                      a->sm_scale, dev_out,
                       dev_lse)))
     return s;
   if ((s = check_host(R, host, dev, host_out, host_lse, dev_lse))) return s;
@@ -463,7 +513,8 @@ dsa_status_t dsa_forward_host(const dsa_layout_t* layout, const dsa_forward_args
   // the key side first: any slab may read any cache row
   ok = ok && copy(a->k_idx, host->k_idx, 0, (size_t)R.n_k * a->D_I * esz, hs) &&
        copy(a->k_scale, host->k_scale, 0, (size_t)R.n_k * 4, hs) &&
-       copy(a->kv, host->kv, 0, (size_t)R.n_k * a->D_K * 2, hs);
+       copy(a->kv, host->kv, 0, (size_t)R.n_k * a->D_K * (a->kv_dtype == DSA_E4M3 ? 1 : 2), hs) &&
+       copy(a->kv_scale, host->kv_scale, 0, (size_t)R.n_k * 4, hs);
   for (int32_t r0 = 0; ok && r0 < R.n_q; r0 += p.slab) {
     const int32_t nr = (R.n_q - r0) < p.slab ? (R.n_q - r0) : p.slab;
     const size_t r = (size_t)r0, n = (size_t)nr;
@@ -474,11 +525,19 @@ dsa_status_t dsa_forward_host(const dsa_layout_t* layout, const dsa_forward_args
          copy(a->q, host->q, r * q_row, n * q_row, hs) && cudaEventRecord(in, hs) == cudaSuccess &&
          cudaStreamWaitEvent(st, in, 0) == cudaSuccess;
     if (!ok) break;
-    if ((s = run_indexer(R, r0, nr, a->idx_dtype, a->H_I, a->D_I, a->q_idx, a->q_scale, a->w,
-                         a->k_idx, a->k_scale, scores, false, st)))
-      break;
-    if ((s = launch_topk(R, r0, nr, scores, R.max_len, a->k, idx, st))) break;
-    if ((s = run_attn(R, r0, nr, a->q, a->kv, idx, a->k, a->H, a->D_K, a->D_V, a->sm_scale,
+    if (p.fused) {
+      if ((s = launch_indexer_select(R, r0, nr, a->idx_dtype, a->H_I, a->D_I, a->q_idx,
+                                     a->q_scale, a->w, a->k_idx, a->k_scale, a->k, idx, scores,
+                                     p.off_idx - p.off_scores, st)))
+        break;
+    } else {
+      if ((s = run_indexer(R, r0, nr, a->idx_dtype, a->H_I, a->D_I, a->q_idx, a->q_scale, a->w,
+                           a->k_idx, a->k_scale, scores, false, st)))
+        break;
+      if ((s = launch_topk(R, r0, nr, scores, R.max_len, a->k, idx, st))) break;
+    }
+    if ((s = run_attn(R, r0, nr, a->q, a->kv, a->kv_scale, idx, a->k, a->H, a->D_K, a->D_V,
+                      a->sm_scale,
                       dev_out, dev_lse, ws + p.off_attn, p.total - p.off_attn, st)))
       break;
     ok = cudaEventRecord(done, st) == cudaSuccess &&

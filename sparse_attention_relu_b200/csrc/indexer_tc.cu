@@ -32,6 +32,7 @@
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
+#include "select.cuh"
 #include "sm100.cuh"
 
 namespace dsa {
@@ -399,7 +400,10 @@ __global__ void __launch_bounds__(kThreadsP, 1)
 // scored).  Equal ranges keep every SM streaming keys until the end, where a
 // grid of per-row chunks paid a prologue and a pipeline ramp per chunk and
 // left the last wave ragged.
-template <int DT, int NK>
+// SEL: the fused selection (top-k) of the decode path; it adds the segment
+// histogram and the ranking scratch of the selection (about 25 KB).
+using SelB = sel::Blk<kEpiThreads, 4, 64>;  // the 512 epilogue threads, named barrier 4
+template <int DT, int NK, bool SEL = false>
 struct DecCfg {
   using C = Cfg<DT, 1, 1, NK>;
   static constexpr int OFF_Q = 0;                         // [2][64 x ROWB] query blocks
@@ -410,10 +414,45 @@ struct DecCfg {
   // k_full/k_empty [NK], s_full/s_empty [NS], q_full/q_empty [2], drain
   static constexpr int NBAR = 2 * NK + 2 * C::NS + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 32 + 1024;
+  static constexpr int OFF_SSM = OFF_MISC + 32;           // sel::Smem (histogram, counters)
+  static constexpr int SSM_BYTES = SEL ? ((int)sizeof(sel::Smem<SelB::NW>) + 15) / 16 * 16 : 0;
+  static constexpr int OFF_CKEY = OFF_SSM + SSM_BYTES;    // [kCand] ranking scratch
+  static constexpr int OFF_CPOS = OFF_CKEY + (SEL ? sel::kCand * 4 : 0);
+  static constexpr int OFF_SELV = OFF_CPOS + (SEL ? sel::kCand * 4 : 0);  // threshold, flag
+  static constexpr int SMEM = OFF_SELV + (SEL ? 16 : 0) + 1024;
   static_assert(C::QBYTES % 1024 == 0 && C::KBYTES % 1024 == 0, "1024-byte operand alignment");
   static_assert(C::NS % kEpiSets == 0, "a TMEM slot always belongs to the same epilogue set");
 };
+
+// The bin that holds the k-th best of the scores a histogram has counted (0
+// while it holds fewer than k): one warp, 64 bins per lane.  The histogram
+// may be read while others still add to it; the counts read are then at
+// most the true ones, which can only lower the bin.
+__device__ __noinline__ uint32_t kth_bin(const uint32_t* hist, int k, int lane) {
+  const volatile uint32_t* h = hist + lane * 64;
+  uint32_t own = 0;
+#pragma unroll 8
+  for (int i = 0; i < 64; ++i) own += h[i];
+  uint32_t suf = own;  // this lane and the lanes above it (higher bins)
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += v;
+  }
+  const uint32_t above = suf - own;
+  uint32_t b = 0;
+  if (above < (uint32_t)k && (uint32_t)k <= suf) {
+    uint32_t c = above;
+    for (int i = 63; i >= 0; --i) {
+      c += h[i];
+      if (c >= (uint32_t)k) {
+        b = (uint32_t)(lane * 64 + i);
+        break;
+      }
+    }
+  }
+  return __reduce_max_sync(0xffffffffu, b);
+}
 
 // Key tiles of decode row r (0 when the row has no candidates).
 __device__ __forceinline__ int32_t dec_row_tiles(const Rows& R, int32_t r) {
@@ -474,14 +513,30 @@ __device__ __forceinline__ bool seg_next(const Rows& R, int32_t row0, int32_t nr
   return false;
 }
 
-template <int DT, int NK>
+// SEL (the fused top-k of dsa_forward's decode path): instead of writing
+// score rows, each score is counted in a histogram of this CTA's segment and
+// kept, as (rank key, position) in its row's candidate list, only when its
+// bin reaches the row's running threshold: the bin of the k-th best score
+// among those counted so far, in this segment or -- shared through a global
+// maximum -- in another CTA's segment of the same row.  The k-th best of any
+// subset of a row is at most the row's k-th best, so no score that can be
+// among the row's k best is dropped ("GLM sparse attention", threshold
+// figure: the cut-off is the k-th best score).  The CTA that finishes the
+// last segment of a row selects the row's top-k from its list.
+//   cand  [nrows][cap] candidates (cap >= max_len, so a list never overflows)
+//   rstate[3][nrows]   per row: candidate count, threshold bin, tiles done
+//                      (zero at launch)
+//   idx   [nrows][k]   the selection, local positions, -1 padded
+template <int DT, int NK, bool SEL = false>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_decode_kernel(const __grid_constant__ CUtensorMap qmap,
                           const __grid_constant__ CUtensorMap kmap, Rows R, int32_t row0,
                           int32_t nrows, const float* __restrict__ w,
                           const float* __restrict__ q_scale, const float* __restrict__ k_scale,
-                          float* __restrict__ scores, int64_t ld, int fill) {
-  using D = DecCfg<DT, NK>;
+                          float* __restrict__ scores, int64_t ld, int fill,
+                          uint64_t* __restrict__ cand, int64_t cap, uint32_t* __restrict__ rstate,
+                          int32_t* __restrict__ idx, int k) {
+  using D = DecCfg<DT, NK, SEL>;
   using C = typename D::C;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -500,6 +555,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + D::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + D::OFF_MISC + 4);
   volatile int32_t* s_first = reinterpret_cast<volatile int32_t*>(smem + D::OFF_MISC + 8);
+  auto* ssm = reinterpret_cast<sel::Smem<SelB::NW>*>(smem + D::OFF_SSM);
+  uint32_t* ckey = reinterpret_cast<uint32_t*>(smem + D::OFF_CKEY);
+  int32_t* cpos = reinterpret_cast<int32_t*>(smem + D::OFF_CPOS);
+  volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(smem + D::OFF_SELV);
+  uint32_t* const rcnt = rstate;              // [nrows] candidates appended
+  uint32_t* const rthr = rstate + nrows;      // [nrows] running threshold bin
+  uint32_t* const rdone = rstate + 2 * nrows;  // [nrows] key tiles scored
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t G = gridDim.x;
 
@@ -511,6 +573,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* o = scores + r * ld;
       for (int32_t s = from + tid; s < R.max_len; s += kThreads) o[s] = -INFINITY;
     }
+  }
+
+  // rows with no candidates at all (fused selection): -1 everywhere
+  if constexpr (SEL) {
+    for (int64_t r = blockIdx.x; r < nrows; r += G)
+      if (dec_row_tiles(R, row0 + (int32_t)r) == 0)
+        for (int i = tid; i < k; i += kThreads) idx[r * k + i] = -1;
   }
 
   // ---- this CTA's share of the concatenated key tiles: [T0, T1)
@@ -558,6 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if constexpr (SEL)
+    for (int i = tid; i < sel::kBins; i += kThreads) ssm->hist[i] = 0;
   if (warp == 1) {
     tmem_alloc(sbase + D::OFF_MISC, C::TCOLS);
     tmem_relinquish();
@@ -693,52 +764,105 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qb = si & 1;
       // warp-uniform outcome of each wait: the tcgen05 loads below need the
       // whole warp, so a lane that gave up takes the others with it
-      if (!__all_sync(0xffffffffu, mbar_wait(q_full(qb), (si >> 1) & 1, R.status) && !*abort_flag)) {
-        ok = false;
-        break;
-      }
+      bool seg_ok =
+          __all_sync(0xffffffffu, mbar_wait(q_full(qb), (si >> 1) & 1, R.status) && !*abort_flag);
       const RowInfo ri = row_info(R, row0 + sg.r);
-      const float4* wr = reinterpret_cast<const float4*>(wq + qb * kHI);
-      float* o = scores + (int64_t)sg.r * ld;
-      // this set's accumulators in the segment: tiles j0, j0 + 4, ...; the key
-      // scales of the next one are fetched while this one is summed (the MMAs
-      // run ahead, so the scale load would otherwise stand alone in the way)
-      const int64_t gt0 = gt;
-      const int j0 = sg.kb + (int)((set - (int)(gt0 % kEpiSets) + kEpiSets) % kEpiSets);
-      auto key_scale = [&](int j) {
-        const int32_t s = j * kTileK + quad * 32 + lane;
-        return (DT == DSA_E4M3 && k_scale && j < sg.ke && s <= ri.t) ? __ldg(k_scale + ri.kbase + s)
-                                                                     : 1.f;
-      };
-      float ks_next = key_scale(j0);
-      gt = gt0 + (sg.ke - sg.kb);
-      for (int j = j0; j < sg.ke; j += kEpiSets) {
-        const int64_t gj = gt0 + (j - sg.kb);
-        const int slot = (int)(gj % C::NS);
-        const int32_t s = j * kTileK + quad * 32 + lane;
-        const float ks = ks_next;
-        ks_next = key_scale(j + kEpiSets);
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(s_full(slot), (int)((gj / C::NS) & 1), R.status) && !*abort_flag)) {
-          ok = false;
-          break;
+      if (seg_ok) {
+        const float4* wr = reinterpret_cast<const float4*>(wq + qb * kHI);
+        float* o = scores + (int64_t)sg.r * ld;
+        // this set's accumulators in the segment: tiles j0, j0 + 4, ...; the key
+        // scales of the next one are fetched while this one is summed (the MMAs
+        // run ahead, so the scale load would otherwise stand alone in the way)
+        const int64_t gt0 = gt;
+        const int j0 = sg.kb + (int)((set - (int)(gt0 % kEpiSets) + kEpiSets) % kEpiSets);
+        auto key_scale = [&](int j) {
+          const int32_t s = j * kTileK + quad * 32 + lane;
+          return (DT == DSA_E4M3 && k_scale && j < sg.ke && s <= ri.t)
+                     ? __ldg(k_scale + ri.kbase + s)
+                     : 1.f;
+        };
+        float ks_next = key_scale(j0);
+        gt = gt0 + (sg.ke - sg.kb);
+        // fused selection: this warp's copy of the row's threshold bin, raised
+        // from the segment histogram every fourth unit and shared through the
+        // row's global maximum
+        uint32_t thr_w = 0, units = 0;
+        if constexpr (SEL) thr_w = __ldcg(rthr + sg.r);
+        for (int j = j0; j < sg.ke; j += kEpiSets) {
+          const int64_t gj = gt0 + (j - sg.kb);
+          const int slot = (int)(gj % C::NS);
+          const int32_t s = j * kTileK + quad * 32 + lane;
+          const float ks = ks_next;
+          ks_next = key_scale(j + kEpiSets);
+          if (!__all_sync(0xffffffffu, mbar_wait(s_full(slot), (int)((gj / C::NS) & 1), R.status) &&
+                                           !*abort_flag)) {
+            seg_ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + slot * C::N;
+          const float sum = relu_wsum(ta, wr);
+          if constexpr (SEL) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_empty(slot));
+            const float x = sum * ks;
+            const bool valid = s <= ri.t;
+            const uint32_t b = sel::score_bin(x);
+            if (valid) atomicAdd(&ssm->hist[b], 1u);
+            const bool keep = valid && b >= thr_w;
+            uint32_t cs;
+            if (sel::warp_append(keep, rcnt + sg.r, cs) && keep)
+              cand[(int64_t)sg.r * cap + cs] = sel::pack_cand(sel::rank_key(x), s);
+            if ((++units & 3) == 0) {
+              const uint32_t bk = kth_bin(ssm->hist, k, lane);
+              uint32_t g = 0;
+              if (lane == 0 && bk > thr_w) g = atomicMax(rthr + sg.r, bk);
+              else if (lane == 0) g = __ldcg(rthr + sg.r);
+              thr_w = max(thr_w, max(bk, __shfl_sync(0xffffffffu, g, 0)));
+            }
+          } else {
+            if (s < R.max_len) {
+              if (s <= ri.t)
+                o[s] = sum * ks;
+              else if (fill)
+                o[s] = -INFINITY;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_empty(slot));
+          }
         }
-        tc_fence_after();
-        const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + slot * C::N;
-        const float sum = relu_wsum(ta, wr);
-        if (s < R.max_len) {
-          if (s <= ri.t)
-            o[s] = sum * ks;
-          else if (fill)
-            o[s] = -INFINITY;
+        if (seg_ok) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(q_empty(qb));
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_empty(slot));
       }
+      if constexpr (SEL) {
+        // every epilogue thread comes here once per segment: the segment's
+        // scores are all counted and filtered (or someone gave up)
+        if (!seg_ok) *abort_flag = 1;
+        seg_ok = bar_red_and<4, kEpiThreads>(seg_ok);
+        if (seg_ok) {
+          const uint32_t seg_tiles = (uint32_t)(sg.ke - sg.kb);
+          const uint32_t row_tiles = (uint32_t)((ri.t + kTileK) / kTileK);
+          if (et == 0) {
+            __threadfence();  // this CTA's candidates before its share of the row's tiles
+            *last_flag = atomicAdd(rdone + sg.r, seg_tiles) + seg_tiles == row_tiles ? 1u : 0u;
+          }
+          asm volatile("bar.sync 4, %0;" ::"n"(kEpiThreads) : "memory");
+          if (*last_flag) {  // the row's last segment: select its k best
+            __threadfence();
+            const uint32_t m = __ldcg(rcnt + sg.r);
+            sel::select_list<SelB>(*ssm, cand + (int64_t)sg.r * cap, m, k,
+                                   idx + (int64_t)sg.r * k, ckey, cpos);
+          }
+          for (int i = et; i < sel::kBins; i += kEpiThreads) ssm->hist[i] = 0;
+          asm volatile("bar.sync 4, %0;" ::"n"(kEpiThreads) : "memory");
+        }
+      }
+      ok = seg_ok;
       if (!ok) break;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_empty(qb));
       ++si;
     } while (seg_next(R, row0, nrows, sg));
     if (!ok) *abort_flag = 1;
@@ -804,12 +928,14 @@ static dsa_status_t launch_cfg(const Rows& R, int32_t row0, int32_t nrows, const
   return launch_status();
 }
 
-template <int DT, int NK>
+// The decode kernel; SEL = the fused selection (cand / rstate / idx / k used).
+template <int DT, int NK, bool SEL = false>
 static dsa_status_t launch_decode(const Rows& R, int32_t row0, int32_t nrows, const void* q_idx,
                                   const float* q_scale, const float* w, const void* k_idx,
                                   const float* k_scale, float* scores, int64_t ld, bool fill,
-                                  cudaStream_t st) {
-  using D = DecCfg<DT, NK>;
+                                  cudaStream_t st, uint64_t* cand = nullptr, int64_t cap = 0,
+                                  uint32_t* rstate = nullptr, int32_t* idx = nullptr, int k = 0) {
+  using D = DecCfg<DT, NK, SEL>;
   using C = typename D::C;
   CUtensorMap qmap, kmap;
   const CUtensorMapDataType tdt =
@@ -818,13 +944,44 @@ static dsa_status_t launch_decode(const Rows& R, int32_t row0, int32_t nrows, co
   if (!make_tmap_2d(&qmap, q_idx, tdt, C::ESZ, kDI, (uint64_t)R.n_q * kHI, box_cols, C::N) ||
       !make_tmap_2d(&kmap, k_idx, tdt, C::ESZ, kDI, (uint64_t)R.n_k, box_cols, kTileK))
     return DSA_ERR_CUDA;
-  auto kfn = indexer_decode_kernel<DT, NK>;
+  auto kfn = indexer_decode_kernel<DT, NK, SEL>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
+  if (SEL && cudaMemsetAsync(rstate, 0, sizeof(uint32_t) * 3 * (size_t)nrows, st) != cudaSuccess)
+    return DSA_ERR_CUDA;
   kfn<<<num_sms(), kThreads, D::SMEM, st>>>(qmap, kmap, R, row0, nrows, w, q_scale, k_scale,
-                                            scores, ld, fill ? 1 : 0);
+                                            scores, ld, fill ? 1 : 0, cand, cap, rstate, idx, k);
   return launch_status();
+}
+
+bool indexer_select_supported(const Rows& R, int dtype, int H_I, int D_I, int k) {
+  return R.mode == DSA_DECODE && indexer_tc_supported(dtype, H_I, D_I) && k >= 1 &&
+         k <= 16384;
+}
+
+size_t indexer_select_workspace(const Rows& R, int32_t nrows) {
+  if (nrows <= 0) return 0;
+  const size_t cand = (size_t)nrows * (size_t)R.max_len * sizeof(uint64_t);
+  return (cand + 255) / 256 * 256 + (size_t)nrows * 3 * sizeof(uint32_t);
+}
+
+dsa_status_t launch_indexer_select(const Rows& R, int32_t row0, int32_t nrows, int dtype,
+                                   int H_I, int D_I, const void* q_idx, const float* q_scale,
+                                   const float* w, const void* k_idx, const float* k_scale, int k,
+                                   int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!indexer_select_supported(R, dtype, H_I, D_I, k)) return DSA_ERR_UNSUPPORTED;
+  if (nrows <= 0) return DSA_OK;
+  if (!ws || ws_bytes < indexer_select_workspace(R, nrows)) return DSA_ERR_WORKSPACE;
+  uint64_t* cand = reinterpret_cast<uint64_t*>(ws);
+  const size_t cbytes = ((size_t)nrows * (size_t)R.max_len * sizeof(uint64_t) + 255) / 256 * 256;
+  uint32_t* rstate = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + cbytes);
+  if (dtype == DSA_BF16)
+    return launch_decode<DSA_BF16, 5, true>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale,
+                                            nullptr, 0, false, st, cand, R.max_len, rstate, idx,
+                                            k);
+  return launch_decode<DSA_E4M3, 11, true>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale,
+                                           nullptr, 0, false, st, cand, R.max_len, rstate, idx, k);
 }
 
 dsa_status_t launch_indexer_tc(const Rows& R, int32_t row0, int32_t nrows, int dtype, int H_I,

@@ -29,6 +29,7 @@
 // ties at the cut filled from the lowest positions by an ordered pass over
 // the row (ballot + warp prefix + a scan of warp totals).
 #include "kernels.cuh"
+#include "select.cuh"
 
 namespace dsa {
 
@@ -36,184 +37,23 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBins = 2048;
-constexpr int kCand = 2048;  // candidate buffer (keys + positions)
+using sel::kBins;
+using sel::kCand;
+using sel::rank_key;
+using sel::score_bin;
+using sel::bin_bounds;
+using sel::warp_append;
+using B512 = sel::Blk<kThreads, 0, 0>;  // the whole CTA, __syncthreads()
+using Smem = sel::Smem<kWarps>;
+__device__ __forceinline__ void find_bin(Smem& sm, int nbins, uint32_t need) {
+  sel::find_bin<B512>(sm, nbins, need);
+}
+__device__ __forceinline__ void rank_candidates(Smem& sm, uint32_t* ckey, int32_t* cpos, int m,
+                                                uint32_t need, int32_t* dst) {
+  sel::rank_candidates<B512>(sm, ckey, cpos, m, need, dst);
+}
 constexpr int kBatch = 4;    // float4 loads each thread keeps in flight per step
 constexpr int kBatchRow = 2;  // the same at three CTAs per SM (42 registers)
-
-__device__ __forceinline__ uint32_t rank_key(float x) {
-  uint32_t u = __float_as_uint(x);
-  if ((u & 0x7fffffffu) > 0x7f800000u) u = 0xff800000u;  // NaN -> -inf
-  if (u == 0x80000000u) u = 0u;                          // -0 -> +0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Bin of a score, 0 .. 2047, non-decreasing in the score: the magnitude
-// bits >> 18 are (exponent, top 5 mantissa bits), clamped to the 1024 steps
-// of 2^-16 .. 2^16; negative scores mirror below 1024.  -0 counts as +0 and
-// NaN as -inf (bin 0).
-constexpr int kMagBase = (111 << 5);  // exponent 111 = 2^-16, mantissa step 0
-__device__ __forceinline__ uint32_t score_bin(float x) {
-  const uint32_t w = __float_as_uint(x), a = w & 0x7fffffffu;
-  const bool neg = w > 0x80000000u || a > 0x7f800000u;
-  const int mb = min(max((int)(a >> 18) - kMagBase, 0), 1023);
-  return neg ? (uint32_t)(1023 - mb) : (uint32_t)(1024 + mb);
-}
-// The floats of bin b form the closed interval [lo, hi].  Bin 0 holds -inf
-// (and NaN, which no float comparison admits); callers handle it apart.
-__device__ __forceinline__ void bin_bounds(uint32_t b, float& lo, float& hi) {
-  const int mb = b >= 1024 ? (int)b - 1024 : 1023 - (int)b;
-  const uint32_t a_lo = mb == 0 ? 0u : (uint32_t)(kMagBase + mb) << 18;
-  const uint32_t a_hi = mb == 1023 ? 0x7f800000u : ((uint32_t)(kMagBase + mb + 1) << 18) - 1u;
-  if (b >= 1024) {
-    lo = __uint_as_float(a_lo);
-    hi = __uint_as_float(a_hi);
-  } else {
-    lo = -__uint_as_float(a_hi);
-    hi = mb == 0 ? -__uint_as_float(1u) : -__uint_as_float(a_lo);  // zeros sit in bin 1024
-  }
-}
-
-struct Smem {
-  uint32_t hist[kBins];
-  uint32_t warp_tot[kWarps];
-  uint32_t sel_bin;
-  uint32_t sel_above;
-  uint32_t n_out;   // positions written so far
-  uint32_t n_cand;  // members of bin b1 seen in pass 2
-  uint32_t kmin, kmax;  // candidate key range (ranking)
-};
-
-// Given hist[0..nbins) and the number `need` of elements still to take,
-// finds bin b with above(b) < need <= above(b) + hist[b], where above(b) is
-// the count in bins > b.  Result in sm.sel_bin / sm.sel_above.
-__device__ void find_bin(Smem& sm, int nbins, uint32_t need) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = nbins / kThreads;  // 4 or 2 contiguous bins per thread
-  const int b0 = tid * per;
-  uint32_t local = 0;
-  for (int i = 0; i < per; ++i) local += sm.hist[b0 + i];
-  // suffix sum over threads: elements in bins owned by higher threads
-  uint32_t incl = local;  // inclusive suffix inside the warp (lanes >= lane)
-  for (int off = 1; off < 32; off <<= 1) {
-    uint32_t v = __shfl_down_sync(0xffffffffu, incl, off);
-    if (lane + off < 32) incl += v;
-  }
-  if (lane == 0) sm.warp_tot[warp] = incl;
-  __syncthreads();
-  uint32_t above = incl - local;
-  for (int w2 = warp + 1; w2 < kWarps; ++w2) above += sm.warp_tot[w2];
-  for (int i = per - 1; i >= 0; --i) {
-    uint32_t h = sm.hist[b0 + i];
-    if (above < need && need <= above + h) {
-      sm.sel_bin = (uint32_t)(b0 + i);
-      sm.sel_above = above;
-    }
-    above += h;
-  }
-  __syncthreads();
-}
-
-// Warp-aggregated append: every lane with `pred` gets a distinct slot of
-// *ctr.  All 32 lanes must call it.
-__device__ __forceinline__ uint32_t warp_append(bool pred, uint32_t* ctr, uint32_t& slot) {
-  const uint32_t mask = __ballot_sync(0xffffffffu, pred);
-  if (!mask) return 0;
-  const int lane = threadIdx.x & 31, leader = __ffs(mask) - 1;
-  uint32_t base = 0;
-  if (lane == leader) base = atomicAdd(ctr, (uint32_t)__popc(mask));
-  base = __shfl_sync(0xffffffffu, base, leader);
-  slot = base + __popc(mask & ((1u << lane) - 1u));
-  return mask;
-}
-
-// Order of candidates: a larger key first, then (the tie rule) the lower
-// position.  Positions are distinct, so no two candidates compare equal.
-__device__ __forceinline__ uint64_t cand_order(uint32_t key, int32_t pos) {
-  return ((uint64_t)key << 32) | (uint64_t)(0xffffffffu - (uint32_t)pos);
-}
-
-__device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-// Writes the `need` best of m <= kCand candidates (key, position) to
-// dst[0 .. need) in any order.  The candidates' keys span [kmin, kmax]; a
-// histogram of (key - kmin) >> shift over kBins buckets (monotone in the key)
-// finds the bucket sb that holds the need-th best.  Candidates in buckets
-// above sb go out at once; the members of sb (typically one or two) move to
-// the front of the candidate arrays and are ranked by the candidate order,
-// one warp per member with its lanes sharing the comparisons, the best of
-// them filling the remaining slots.  All threads of the CTA call it.
-__device__ void rank_candidates(Smem& sm, uint32_t* ckey, int32_t* cpos, int m, uint32_t need,
-                                int32_t* dst) {
-  constexpr int R = kCand / kThreads;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t key[R];
-  int32_t pos[R];
-  uint32_t lo = 0xffffffffu, hi = 0u;
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int j = tid + r * kThreads;
-    key[r] = j < m ? ckey[j] : 0u;
-    pos[r] = j < m ? cpos[j] : 0;
-    if (j < m) {
-      lo = min(lo, key[r]);
-      hi = max(hi, key[r]);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-  }
-  if (tid == 0) {
-    sm.kmin = 0xffffffffu;
-    sm.kmax = 0u;
-    sm.n_out = 0;
-    sm.n_cand = 0;
-  }
-  for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0;
-  __syncthreads();
-  if (lane == 0) {
-    atomicMin(&sm.kmin, lo);
-    atomicMax(&sm.kmax, hi);
-  }
-  __syncthreads();
-  const uint32_t kmin = sm.kmin, span = sm.kmax - kmin;
-  const int bits = span ? 32 - __clz(span) : 0;  // bits of the span
-  const int shift = bits > 11 ? bits - 11 : 0;   // (span >> shift) < 2048 buckets
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-    if (tid + r * kThreads < m) atomicAdd(&sm.hist[(key[r] - kmin) >> shift], 1u);
-  __syncthreads();
-  find_bin(sm, kBins, need);  // ends with a barrier: every candidate is in registers
-  const uint32_t sb = sm.sel_bin, need2 = need - sm.sel_above;
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const bool ok = tid + r * kThreads < m;
-    const uint32_t b = (key[r] - kmin) >> shift;
-    const bool up = ok && b > sb, in = ok && b == sb;
-    uint32_t slot;
-    if (warp_append(up, &sm.n_out, slot) && up) dst[slot] = pos[r];
-    if (warp_append(in, &sm.n_cand, slot) && in) {
-      ckey[slot] = key[r];
-      cpos[slot] = pos[r];
-    }
-  }
-  __syncthreads();
-  const int c = (int)sm.n_cand;
-  const uint32_t base_out = sm.n_out;  // == sm.sel_above
-  for (int j = warp; j < c; j += kWarps) {
-    const uint64_t oj = cand_order(ckey[j], cpos[j]);
-    uint32_t better = 0;
-    for (int l = lane; l < c; l += 32) better += cand_order(ckey[l], cpos[l]) > oj ? 1u : 0u;
-    better = warp_sum(better);
-    if (lane == 0 && better < need2) dst[base_out + better] = cpos[j];
-  }
-}
 
 // The members of bin b1 (more than the candidate buffer holds) resolved from
 // the row itself: three radix levels over their fp32 keys find the k-th key

@@ -49,7 +49,12 @@ class Dev:
         lse = torch.empty(wl.n_q, c.H, dtype=torch.float32, device="cuda")
         nws = dsa.dsa_sparse_mla_attn_workspace_size(self.layout, k, c.H, c.D_K, c.D_V)
         ws = torch.empty(max(nws, 16), dtype=torch.uint8, device="cuda")
-        dsa.dsa_sparse_mla_attn(self.layout, d.q, d.kv, idx, k, c.D_V, c.sm_scale, out, lse, ws)
+        if d.kv_scale is not None:  # FP8 cache
+            dsa.dsa_sparse_mla_attn_e4m3(self.layout, d.q, d.kv, d.kv_scale, idx, k, c.D_V,
+                                         c.sm_scale, out, lse, ws)
+        else:
+            dsa.dsa_sparse_mla_attn(self.layout, d.q, d.kv, idx, k, c.D_V, c.sm_scale, out, lse,
+                                    ws)
         return out, lse
 
     def forward(self, with_idx=True):
@@ -57,7 +62,7 @@ class Dev:
         c = wl.cfg
         args = dsa.forward_args(q_idx=d.q_idx, q_scale=d.q_scale, w=d.w, k_idx=d.k_idx,
                                 k_scale=d.k_scale, q=d.q, kv=d.kv, D_V=c.D_V,
-                                sm_scale=c.sm_scale, k=c.k)
+                                sm_scale=c.sm_scale, k=c.k, kv_scale=d.kv_scale)
         nws = dsa.dsa_forward_workspace_size(self.layout, args)
         ws = torch.empty(max(nws, 16), dtype=torch.uint8, device="cuda")
         out = torch.empty(wl.n_q, c.H, c.D_V, dtype=torch.bfloat16, device="cuda")

@@ -78,6 +78,12 @@ def test_argument_validation_without_device(lib):
     assert f(ctypes.byref(L), P, P, P, 4, 129, 576, 512, 0.1, P, None, None, 0, None) == E
     assert f(ctypes.byref(L), P, P, P, 4, 128, 576, 580, 0.1, P, None, None, 0, None) == E
     assert f(ctypes.byref(L), P, P, P, 4, 8, 80, 64, float("nan"), P, None, None, 0, None) == E
+    # attention over an FP8 cache: scales required and aligned, D_K a multiple of 16
+    g = lib.dsa_sparse_mla_attn_e4m3
+    assert g(ctypes.byref(L), P, P, None, P, 4, 8, 80, 64, 0.1, P, None, None, 0, None) == E
+    assert g(ctypes.byref(L), P, P, P + 4, P, 4, 8, 80, 64, 0.1, P, None, None, 0, None) == E
+    assert g(ctypes.byref(L), P, P, P, P, 4, 8, 72, 64, 0.1, P, None, None, 0, None) == E
+    assert g(ctypes.byref(L), P, P, P, P, 0, 8, 80, 64, 0.1, P, None, None, 0, None) == E
     # chunked prefill: query offsets required, and no more queries than cache rows
     ch = _layout(mode=dsa.DSA_CHUNKED, n_q=4)
     assert lib.dsa_topk(ctypes.byref(ch), P, 4, P, None) == E  # q_offsets missing
@@ -107,7 +113,7 @@ def test_forward_host_validation_without_device(lib):
     def args(ptr, **kw):
         d = dict(idx_dtype=dsa.DSA_BF16, H_I=64, D_I=128, q_idx=ptr, q_scale=None, w=ptr,
                  k_idx=ptr, k_scale=None, H=128, D_K=576, D_V=512, sm_scale=0.1, q=ptr, kv=ptr,
-                 k=4)
+                 k=4, kv_dtype=dsa.DSA_BF16, kv_scale=None)
         d.update(kw)
         return dsa.dsa_forward_args_t(*d.values())
 
@@ -128,6 +134,11 @@ def test_forward_host_validation_without_device(lib):
     assert call(args(H), host_lse=H) == E  # host lse without a device lse
     e4 = args(P, idx_dtype=dsa.DSA_E4M3, q_scale=P, k_scale=P)
     assert call(args(H, idx_dtype=dsa.DSA_E4M3, k_scale=H), dev_args=e4) == E  # q_scale missing
+    # FP8 MLA cache: the host block's cache type must match; a bf16 cache has no scales
+    f8 = args(P, kv_dtype=dsa.DSA_E4M3, kv_scale=P)
+    assert call(args(H), dev_args=f8) == E
+    assert call(args(H, kv_scale=H)) == E
+    assert call(args(H, kv_dtype=dsa.DSA_E4M3, kv_scale=H), dev_args=args(P, kv_dtype=dsa.DSA_E4M3)) == E
     assert lib.dsa_forward_host_workspace_size(ctypes.byref(L), ctypes.byref(dev), -1) == 0
 
 

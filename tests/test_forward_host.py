@@ -28,15 +28,17 @@ def _host_call(dev, rows_per_slab=0, resident=False, pin=True, with_lse=True):
             return None
         return t.contiguous().pin_memory() if pin else t.contiguous()
 
+    kv_dtype = dsa.DSA_E4M3 if d.kv_scale is not None else dsa.DSA_BF16
     host = dsa.forward_args(q_idx=h(wl.q_idx), q_scale=h(wl.q_scale), w=h(wl.w),
                             k_idx=None if resident else h(wl.k_idx),
                             k_scale=None if resident else h(wl.k_scale), q=h(wl.q),
                             kv=None if resident else h(wl.kv), D_V=c.D_V, sm_scale=c.sm_scale,
-                            k=c.k, host=True)
+                            k=c.k, host=True,
+                            kv_scale=None if resident else h(wl.kv_scale), kv_dtype=kv_dtype)
     # device buffers: queries start as garbage; the cache is current only when resident
     bufs = {n: torch.empty_like(getattr(d, n)) for n in ("q_idx", "w", "q")}
     bufs["q_scale"] = None if d.q_scale is None else torch.empty_like(d.q_scale)
-    for n in ("k_idx", "k_scale", "kv"):
+    for n in ("k_idx", "k_scale", "kv", "kv_scale"):
         t = getattr(d, n)
         bufs[n] = None if t is None else (t.clone() if resident else torch.zeros_like(t))
     devargs = dsa.forward_args(D_V=c.D_V, sm_scale=c.sm_scale, k=c.k, **bufs)
@@ -70,9 +72,9 @@ def _check(dev, out_h, lse_h, ref, idx, n_sample=None, must=()):
                       o_dev[rows].float().cpu().numpy(), l_dev[rows].cpu().numpy())
 
 
-def _prefill():
+def _prefill(kv_dtype="bf16"):
     return Dev(workloads.generate(workloads.custom("prefill", [700, 300], idx_dtype="e4m3", k=64,
-                                                   seed=11)))
+                                                   seed=11, kv_dtype=kv_dtype)))
 
 
 def test_default_slabs_match_forward_and_oracle():
@@ -83,24 +85,40 @@ def test_default_slabs_match_forward_and_oracle():
     _check(dev, out_h, lse_h, (out, lse), idx, n_sample=32)
 
 
-@pytest.mark.parametrize("pin", [True, False])
-def test_small_slabs_match_forward_and_oracle(pin):
-    """256-row slabs over 1000 queries: four slabs, the last one 232 rows."""
-    dev = _prefill()
+@pytest.mark.parametrize("pin,kv_dtype", [(True, "bf16"), (False, "bf16"), (True, "e4m3")])
+def test_small_slabs_match_forward_and_oracle(pin, kv_dtype):
+    """256-row slabs over 1000 queries: four slabs, the last one 232 rows
+    (with a bf16 MLA cache, and with an FP8 one whose scales travel too)."""
+    dev = _prefill(kv_dtype)
     out, lse, idx = dev.forward()
     out_h, lse_h = _host_call(dev, rows_per_slab=256, pin=pin)
     assert dev.status() == dsa.DSA_OK
     _check(dev, out_h, lse_h, (out, lse), idx, n_sample=24, must=[255, 256, 511, 767, 768])
 
 
-@pytest.mark.parametrize("mode,lens", [("decode", [700, 300, 129]),
-                                       ("chunked", [900, 400])])
-def test_resident_cache_matches_forward_and_oracle(mode, lens):
+@pytest.mark.parametrize("mode,lens,kv_dtype", [("decode", [700, 300, 129], "bf16"),
+                                                ("chunked", [900, 400], "bf16"),
+                                                ("decode", [700, 300, 129], "e4m3")])
+def test_resident_cache_matches_forward_and_oracle(mode, lens, kv_dtype):
     kw = dict(chunks=[128, 64]) if mode == "chunked" else {}
     dev = Dev(workloads.generate(workloads.custom(mode, lens, idx_dtype="bf16", k=128, seed=3,
-                                                  **kw)))
+                                                  kv_dtype=kv_dtype, **kw)))
     out, lse, idx = dev.forward()
     out_h, lse_h = _host_call(dev, resident=True)
+    assert dev.status() == dsa.DSA_OK
+    _check(dev, out_h, lse_h, (out, lse), idx)
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "e4m3"])
+def test_decode_in_slabs_of_rows(kv_dtype):
+    """Decode through dsa_forward_host in slabs of 16 rows: every kernel of the
+    path (the persistent decode indexer, the split top-k, the split attention
+    and its merge) starts at a row offset, with the caches resident."""
+    lens = [3000 + 977 * i for i in range(37)]
+    dev = Dev(workloads.generate(workloads.custom("decode", lens, idx_dtype="e4m3", k=2048,
+                                                  seed=17, kv_dtype=kv_dtype)))
+    out, lse, idx = dev.forward()
+    out_h, lse_h = _host_call(dev, rows_per_slab=16, resident=True)
     assert dev.status() == dsa.DSA_OK
     _check(dev, out_h, lse_h, (out, lse), idx)
 
