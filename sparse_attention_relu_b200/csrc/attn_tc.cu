@@ -78,7 +78,7 @@ constexpr int kStages = 2;
 constexpr int kAtomsA = 5, kAtomsV = 4;
 constexpr int kChunksA = kNT * kAtomsA * 8;    // 2560 16-byte chunks
 constexpr int kChunksV = kNT * kAtomsV * 8;    // 2048
-constexpr int kIdxRing = 4;                    // tiles whose indices are held
+constexpr int kIdxRing = 8;                    // tiles whose indices are held
 // e4m3 cache: a 16-byte load brings 16 codes, two 16-byte bf16 chunks of the
 // swizzled operand, so each group takes half as many loads as chunks.
 constexpr int kLoadsA = kChunksA / 2, kLoadsV = kChunksV / 2;  // 1280, 1024
@@ -94,7 +94,7 @@ constexpr int OFF_MASK = OFF_IDX + kIdxRing * kNT * 4;   // [ring][2] uint32 val
 constexpr int OFF_HMAX = OFF_MASK + kIdxRing * 2 * 4;    // [2 tiles][2 warpgroups][128] float
 constexpr int OFF_KSC = OFF_HMAX + 2 * 2 * kH * 4;       // [ring][64] fp32 cache scales (e4m3)
 constexpr int OFF_BAR = OFF_KSC + kIdxRing * kNT * 4;
-constexpr int kNumBars = 18;
+constexpr int kNumBars = 22;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 // The dynamic window starts 1024-aligned (right after the driver's reserved
 // kilobyte, with no static shared memory); the kernel checks it.
@@ -106,10 +106,11 @@ constexpr uint32_t TM_Q = 0;     // query dims 0..383 of all heads, bf16 pairs (
 constexpr uint32_t TM_S = 192;   // 64-column score tile
 constexpr uint32_t TM_O = 256;   // 256-column output accumulator
 constexpr uint32_t IDESC_QK = idesc(1, 128, kNT);
-// PV runs as N = 64 MMAs (one per 64 value columns): the QK MMAs are N = 64,
-// and a stream that mixes MMA shapes was measured on B200 to take about twice
-// the time of its parts.
-constexpr int kPvN = 64;
+// PV MMA width: 256 (one MMA per 16 rows of the tile for this CTA's value
+// columns).  Four N = 64 MMAs instead (the QK MMAs are N = 64; a probe stream
+// that mixed N = 64 and N = 256 MMAs took about twice the time of its parts)
+// measured 3% slower in this kernel.
+constexpr int kPvN = 256;
 constexpr uint32_t IDESC_PV = idesc(1, 128, kPvN, false, true);
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -361,87 +362,114 @@ __global__ void __launch_bounds__(kThreads, 1)
                    "r"(nbytes)
                    : "memory");
     };
-    for (int n = 0; n < ntiles; ++n) {
-      const int st = n % kStages, ring = n % kIdxRing;
-      const uint32_t par = ((n / kStages) & 1) ^ 1;
-      // group A of the stage is free once QK(n-2) read it
-      bool ok = mbar_wait(bar(B_AEMPTY + st), par, R.status) && !*abort_flag;
-      if (!bar_and<2, kProducers>(ok)) {
-        *abort_flag = 1;
-        break;
-      }
+    // Publishes the indices (and mask and scales) of tile n into ring slot
+    // n % kIdxRing (threads 0..63 hold them in pre / pre_sc), then loads tile
+    // n+1's into pre / pre_sc.
+    auto publish = [&](int n) {
+      const int ring = n % kIdxRing;
       if (tid < kNT) {
         sidx[ring * kNT + tid] = pre;
         if (FP8) ksc[ring * kNT + tid] = pre_sc;
         const uint32_t bits = __ballot_sync(0xffffffffu, pre >= 0);
         if (lane == 0) vmask[ring * 2 + warp] = bits;
       }
-      mbar_arrive(bar(B_AFULL + st));   // publishes indices to the MMA issuer
-      mbar_arrive(bar(B_IDX + ring));   // ... and indices, mask, scales to the softmax threads
-      asm volatile("bar.sync 2, %0;" ::"n"(kProducers) : "memory");  // producers see the indices
+      mbar_arrive(bar(B_AFULL + n % kStages));  // publishes indices to the MMA issuer
+      mbar_arrive(bar(B_IDX + ring));           // ... and indices, mask, scales to the softmax
+      asm volatile("bar.sync 2, %0;" ::"n"(kProducers) : "memory");  // producers see them
       if (tid < kNT) {  // overlaps the copies below
         pre = n + 1 < ntiles ? load_idx(n + 1) : -1;
         pre_sc = load_scale(pre);
       }
-      if constexpr (FP8) {
-        // group A through registers: all loads in flight, then convert and store
-        constexpr int J = (kLoadsA + kProducers - 1) / kProducers;
-        uint4 x[J];
+    };
+    if constexpr (FP8) {
+      // Codes go through registers (converted on the way into the swizzled
+      // bf16 operand), software-pipelined: tile n+1's loads are in flight
+      // while tile n waits for its stage, which QK(n-2) and PV(n-2) release.
+      constexpr int JA = (kLoadsA + kProducers - 1) / kProducers;
+      constexpr int JV = (kLoadsV + kProducers - 1) / kProducers;
+      uint4 xa[JA], xv[JV];
+      auto load = [&](int n) {
+        const int ring = n % kIdxRing;
 #pragma unroll
-        for (int j = 0; j < J; ++j) {
+        for (int j = 0; j < JA; ++j) {
           const int i = tid + kProducers * j, c = i & 3, seg = i >> 2, row = seg / kAtomsA;
           const int ai = seg - row * kAtomsA, atom = ai < 4 ? 4 * (half ^ 1) + ai : 8;
           const int32_t s = i < kLoadsA ? sidx[ring * kNT + row] : -1;
-          x[j] = s >= 0 ? ld_nc_v4(kvb + (int64_t)s * kRowBytes + atom * 64 + c * 16)
-                        : make_uint4(0, 0, 0, 0);
+          xa[j] = s >= 0 ? ld_nc_v4(kvb + (int64_t)s * kRowBytes + atom * 64 + c * 16)
+                         : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int j = 0; j < J; ++j) {
+        for (int j = 0; j < JV; ++j) {  // 16 codes per load: quarter c of segment (row, atom)
+          const int i = tid + kProducers * j, c = i & 3, seg = i >> 2, row = seg >> 2;
+          const int atom = 4 * half + (seg & 3);
+          const int32_t s = i < kLoadsV ? sidx[ring * kNT + row] : -1;
+          xv[j] = s >= 0 ? ld_nc_v4(kvb + (int64_t)s * kRowBytes + atom * 64 + c * 16)
+                         : make_uint4(0, 0, 0, 0);
+        }
+      };
+      if (ntiles > 0) {
+        publish(0);
+        load(0);
+      }
+      for (int n = 0; n < ntiles; ++n) {
+        const int st = n % kStages;
+        const uint32_t par = ((n / kStages) & 1) ^ 1;
+        bool ok = mbar_wait(bar(B_AEMPTY + st), par, R.status) &&
+                  mbar_wait(bar(B_VEMPTY + st), par, R.status) && !*abort_flag;
+        if (!bar_and<2, kProducers>(ok)) {
+          *abort_flag = 1;
+          break;
+        }
+#pragma unroll
+        for (int j = 0; j < JA; ++j) {
           const int i = tid + kProducers * j, c = i & 3, seg = i >> 2, row = seg / kAtomsA;
           const int ai = seg - row * kAtomsA, atom = ai < 4 ? 4 * (half ^ 1) + ai : 8;
           if (i < kLoadsA)
-            store_codes(smem + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128, c, row, x[j]);
+            store_codes(smem + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128, c, row,
+                        xa[j]);
         }
         fence_async_smem();
         mbar_arrive(bar(B_AFULL + st));
-      } else {
+#pragma unroll
+        for (int j = 0; j < JV; ++j) {
+          const int i = tid + kProducers * j, c = i & 3, seg = i >> 2, row = seg >> 2;
+          const int atom = 4 * half + (seg & 3);
+          if (i < kLoadsV)
+            store_codes(smem + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128, c, row,
+                        xv[j]);
+        }
+        fence_async_smem();
+        mbar_arrive(bar(B_VFULL + st));
+        if (n + 1 < ntiles) {
+          publish(n + 1);
+          load(n + 1);
+        }
+      }
+    } else {
+      for (int n = 0; n < ntiles; ++n) {
+        const int st = n % kStages, ring = n % kIdxRing;
+        const uint32_t par = ((n / kStages) & 1) ^ 1;
+        // group A of the stage is free once QK(n-2) read it
+        bool ok = mbar_wait(bar(B_AEMPTY + st), par, R.status) && !*abort_flag;
+        if (!bar_and<2, kProducers>(ok)) {
+          *abort_flag = 1;
+          break;
+        }
+        publish(n);
 #pragma unroll
         for (int j = 0; j < (kChunksA + kProducers - 1) / kProducers; ++j)
           if (tid + kProducers * j < kChunksA) issue(st, ring, tid + kProducers * j, true);
         asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
                          bar(B_AFULL + st))
                      : "memory");
-      }
-      // group V of the stage (this CTA's value columns) is free once PV(n-2)
-      // read it; the producers fetch it too, so that the softmax threads never
-      // wait for a PV to retire
-      ok = mbar_wait(bar(B_VEMPTY + st), par, R.status) && !*abort_flag;
-      if (!bar_and<2, kProducers>(ok)) {
-        *abort_flag = 1;
-        break;
-      }
-      if constexpr (FP8) {
-        // 16 codes per load: segment (row, atom) quarter c holds dims 16c .. 16c+15
-        constexpr int J = (kLoadsV + kProducers - 1) / kProducers;
-        uint4 x[J];
-#pragma unroll
-        for (int j = 0; j < J; ++j) {
-          const int i = tid + kProducers * j, c = i & 3, seg = i >> 2, row = seg >> 2;
-          const int atom = 4 * half + (seg & 3);
-          const int32_t s = i < kLoadsV ? sidx[ring * kNT + row] : -1;
-          x[j] = s >= 0 ? ld_nc_v4(kvb + (int64_t)s * kRowBytes + atom * 64 + c * 16)
-                        : make_uint4(0, 0, 0, 0);
+        // group V of the stage (this CTA's value columns) is free once PV(n-2)
+        // read it; the producers fetch it too, so that the softmax threads
+        // never wait for a PV to retire
+        ok = mbar_wait(bar(B_VEMPTY + st), par, R.status) && !*abort_flag;
+        if (!bar_and<2, kProducers>(ok)) {
+          *abort_flag = 1;
+          break;
         }
-#pragma unroll
-        for (int j = 0; j < J; ++j) {
-          const int i = tid + kProducers * j, c = i & 3, seg = i >> 2, row = seg >> 2;
-          const int atom = 4 * half + (seg & 3);
-          if (i < kLoadsV)
-            store_codes(smem + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128, c, row, x[j]);
-        }
-        fence_async_smem();
-        mbar_arrive(bar(B_VFULL + st));
-      } else {
 #pragma unroll
         for (int j = 0; j < (kChunksV + kProducers - 1) / kProducers; ++j)
           if (tid + kProducers * j < kChunksV) issue(st, ring, tid + kProducers * j, false);
@@ -616,9 +644,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = n % kStages;
       float s[32];
       // S(n) retired; then the tile's validity bits and scales are visible
-      // (B_IDX: the producers published them; they cannot publish tile n+4
-      // into this slot before this thread has read S(n+1), so the parity
-      // names tile n's phase)
+      // (B_IDX: the producers published them; they cannot publish tile
+      // n + kIdxRing into this slot before this thread has read S(n+1), so
+      // the parity names tile n's phase)
       bool w_ok = __all_sync(0xffffffffu,
                              mbar_wait(bar(B_SFULL), n & 1, R.status) &&
                                  mbar_wait(bar(B_IDX + n % kIdxRing), (n / kIdxRing) & 1,

@@ -107,6 +107,26 @@ __device__ __forceinline__ float relu_wsum(uint32_t ta, const float4* __restrict
          ((lo32(acc[2]) + hi32(acc[2])) + (lo32(acc[3]) + hi32(acc[3])));
 }
 
+// relu_wsum with one 32-column TMEM load at a time.
+__device__ __forceinline__ float relu_wsum_halves(uint32_t ta, const float4* __restrict__ wr) {
+  uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float v[32];
+    tmem_ld32(ta + 32 * half, v);
+#pragma unroll
+    for (int h4 = 0; h4 < 8; ++h4) {
+      const float4 w4 = wr[8 * half + h4];
+      acc[(2 * h4) & 3] = fma2(fmaxf(v[4 * h4], 0.f), fmaxf(v[4 * h4 + 1], 0.f), w4.x, w4.y,
+                               acc[(2 * h4) & 3]);
+      acc[(2 * h4 + 1) & 3] = fma2(fmaxf(v[4 * h4 + 2], 0.f), fmaxf(v[4 * h4 + 3], 0.f), w4.z,
+                                   w4.w, acc[(2 * h4 + 1) & 3]);
+    }
+  }
+  return (lo32(acc[0]) + hi32(acc[0])) + (lo32(acc[1]) + hi32(acc[1])) +
+         ((lo32(acc[2]) + hi32(acc[2])) + (lo32(acc[3]) + hi32(acc[3])));
+}
+
 template <int DT, int G, int NG, int NK>
 struct Cfg {
   static constexpr int ESZ = DT == DSA_BF16 ? 2 : 1;
@@ -400,8 +420,8 @@ __global__ void __launch_bounds__(kThreadsP, 1)
 // scored).  Equal ranges keep every SM streaming keys until the end, where a
 // grid of per-row chunks paid a prologue and a pipeline ramp per chunk and
 // left the last wave ragged.
-// SEL: the fused selection (top-k) of the decode path; it adds the segment
-// histogram and the ranking scratch of the selection (about 25 KB).
+// SEL: the fused filter of the decode path; it adds the segment histogram
+// (8 KB) and the segment's candidate counter.
 using SelB = sel::Blk<kEpiThreads, 4, 64>;  // the 512 epilogue threads, named barrier 4
 template <int DT, int NK, bool SEL = false>
 struct DecCfg {
@@ -414,44 +434,56 @@ struct DecCfg {
   // k_full/k_empty [NK], s_full/s_empty [NS], q_full/q_empty [2], drain
   static constexpr int NBAR = 2 * NK + 2 * C::NS + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int OFF_SSM = OFF_MISC + 32;           // sel::Smem (histogram, counters)
+  static constexpr int OFF_SSM = (OFF_MISC + 32 + 15) / 16 * 16;  // sel::Smem (histogram first)
   static constexpr int SSM_BYTES = SEL ? ((int)sizeof(sel::Smem<SelB::NW>) + 15) / 16 * 16 : 0;
-  static constexpr int OFF_CKEY = OFF_SSM + SSM_BYTES;    // [kCand] ranking scratch
-  static constexpr int OFF_CPOS = OFF_CKEY + (SEL ? sel::kCand * 4 : 0);
-  static constexpr int OFF_SELV = OFF_CPOS + (SEL ? sel::kCand * 4 : 0);  // threshold, flag
-  static constexpr int SMEM = OFF_SELV + (SEL ? 16 : 0) + 1024;
+  static constexpr int OFF_SCNT = OFF_SSM + SSM_BYTES;     // the segment's candidate count
+  static constexpr int SMEM = OFF_SCNT + (SEL ? 16 : 0) + 1024;
   static_assert(C::QBYTES % 1024 == 0 && C::KBYTES % 1024 == 0, "1024-byte operand alignment");
   static_assert(C::NS % kEpiSets == 0, "a TMEM slot always belongs to the same epilogue set");
 };
 
 // The bin that holds the k-th best of the scores a histogram has counted (0
-// while it holds fewer than k): one warp, 64 bins per lane.  The histogram
-// may be read while others still add to it; the counts read are then at
-// most the true ones, which can only lower the bin.
+// while it holds fewer than k): one warp.  Each lane sums 64 bins (16-byte
+// loads), a suffix scan over the lanes finds the lane whose bins hold the
+// k-th best, and a second scan over that lane's bins, two per lane, finds
+// the bin.  The histogram may be read while others still add to it; the
+// counts read are then at most the true ones, which can only lower the bin.
 __device__ __noinline__ uint32_t kth_bin(const uint32_t* hist, int k, int lane) {
-  const volatile uint32_t* h = hist + lane * 64;
+  const uint4* h4 = reinterpret_cast<const uint4*>(hist) + lane * 16;
   uint32_t own = 0;
-#pragma unroll 8
-  for (int i = 0; i < 64; ++i) own += h[i];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint4 v = h4[i];
+    own += (v.x + v.y) + (v.z + v.w);
+  }
   uint32_t suf = own;  // this lane and the lanes above it (higher bins)
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
     if (lane + o < 32) suf += v;
   }
-  const uint32_t above = suf - own;
-  uint32_t b = 0;
-  if (above < (uint32_t)k && (uint32_t)k <= suf) {
-    uint32_t c = above;
-    for (int i = 63; i >= 0; --i) {
-      c += h[i];
-      if (c >= (uint32_t)k) {
-        b = (uint32_t)(lane * 64 + i);
-        break;
-      }
-    }
+  const uint32_t kk = (uint32_t)k;
+  const uint32_t hit = __ballot_sync(0xffffffffu, suf - own < kk && kk <= suf);
+  if (!hit) return 0u;
+  const int L = __ffs(hit) - 1;
+  const uint32_t need = kk - __shfl_sync(0xffffffffu, suf - own, L);  // 1 .. lane L's count
+  // lane L's 64 bins, two per lane (bins 2j, 2j+1 of the 64), counted from the top
+  const uint2 c = reinterpret_cast<const uint2*>(hist + L * 64)[lane];
+  const uint32_t pair = c.x + c.y;
+  uint32_t sp = pair;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xffffffffu, sp, o);
+    if (lane + o < 32) sp += v;
   }
-  return __reduce_max_sync(0xffffffffu, b);
+  const uint32_t above = sp - pair;  // in higher bins of lane L's 64
+  const bool in_hi = above < need && need <= above + c.y;
+  const bool in_lo = !in_hi && above + c.y < need && need <= sp;
+  const uint32_t bh = __ballot_sync(0xffffffffu, in_hi || in_lo);
+  if (!bh) return 0u;  // (cannot happen: counts only grow between the two reads)
+  const int j = __ffs(bh) - 1;
+  const uint32_t hi_bit = __shfl_sync(0xffffffffu, in_hi ? 1u : 0u, j);
+  return (uint32_t)(L * 64 + 2 * j) + hi_bit;
 }
 
 // Key tiles of decode row r (0 when the row has no candidates).
@@ -521,12 +553,16 @@ __device__ __forceinline__ bool seg_next(const Rows& R, int32_t row0, int32_t nr
 // maximum -- in another CTA's segment of the same row.  The k-th best of any
 // subset of a row is at most the row's k-th best, so no score that can be
 // among the row's k best is dropped ("GLM sparse attention", threshold
-// figure: the cut-off is the k-th best score).  The CTA that finishes the
-// last segment of a row selects the row's top-k from its list.
-//   cand  [nrows][cap] candidates (cap >= max_len, so a list never overflows)
-//   rstate[3][nrows]   per row: candidate count, threshold bin, tiles done
-//                      (zero at launch)
-//   idx   [nrows][k]   the selection, local positions, -1 padded
+// figure: the cut-off is the k-th best score).  A segment over the row's key
+// tiles [kb, ke) appends to its own part of the row's list, entries
+// kb*128 .. ke*128 (so no list overflows and no two CTAs share a counter),
+// and at its end records its count and adds its histogram into the row's;
+// select_rows_kernel then picks each row's k best from its segments' lists.
+//   cand  [nrows][cap]        candidates (cap >= max_len)
+//   rstate[nrows]             per row: running threshold bin (zero at launch)
+//   segcnt[nrows][cap / 128]  per row and first tile of a segment: its
+//                             candidate count (zero at launch)
+//   rhist [nrows][kBins]      per row: histogram of all its scores (zero at launch)
 template <int DT, int NK, bool SEL = false>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_decode_kernel(const __grid_constant__ CUtensorMap qmap,
@@ -535,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const float* __restrict__ q_scale, const float* __restrict__ k_scale,
                           float* __restrict__ scores, int64_t ld, int fill,
                           uint64_t* __restrict__ cand, int64_t cap, uint32_t* __restrict__ rstate,
-                          int32_t* __restrict__ idx, int k) {
+                          uint32_t* __restrict__ segcnt, uint32_t* __restrict__ rhist, int k) {
   using D = DecCfg<DT, NK, SEL>;
   using C = typename D::C;
   extern __shared__ uint8_t smem_raw[];
@@ -556,12 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + D::OFF_MISC + 4);
   volatile int32_t* s_first = reinterpret_cast<volatile int32_t*>(smem + D::OFF_MISC + 8);
   auto* ssm = reinterpret_cast<sel::Smem<SelB::NW>*>(smem + D::OFF_SSM);
-  uint32_t* ckey = reinterpret_cast<uint32_t*>(smem + D::OFF_CKEY);
-  int32_t* cpos = reinterpret_cast<int32_t*>(smem + D::OFF_CPOS);
-  volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(smem + D::OFF_SELV);
-  uint32_t* const rcnt = rstate;              // [nrows] candidates appended
-  uint32_t* const rthr = rstate + nrows;      // [nrows] running threshold bin
-  uint32_t* const rdone = rstate + 2 * nrows;  // [nrows] key tiles scored
+  uint32_t* const rthr = rstate;  // [nrows] running threshold bin
+  uint32_t* const scnt = reinterpret_cast<uint32_t*>(smem + D::OFF_SCNT);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t G = gridDim.x;
 
@@ -573,13 +605,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* o = scores + r * ld;
       for (int32_t s = from + tid; s < R.max_len; s += kThreads) o[s] = -INFINITY;
     }
-  }
-
-  // rows with no candidates at all (fused selection): -1 everywhere
-  if constexpr (SEL) {
-    for (int64_t r = blockIdx.x; r < nrows; r += G)
-      if (dec_row_tiles(R, row0 + (int32_t)r) == 0)
-        for (int i = tid; i < k; i += kThreads) idx[r * k + i] = -1;
   }
 
   // ---- this CTA's share of the concatenated key tiles: [T0, T1)
@@ -627,8 +652,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if constexpr (SEL)
+  if constexpr (SEL) {
     for (int i = tid; i < sel::kBins; i += kThreads) ssm->hist[i] = 0;
+    if (tid == 0) *scnt = 0;
+  }
   if (warp == 1) {
     tmem_alloc(sbase + D::OFF_MISC, C::TCOLS);
     tmem_relinquish();
@@ -801,7 +828,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + slot * C::N;
-          const float sum = relu_wsum(ta, wr);
+          // (the fused filter reads the 64 head scores 32 at a time: fewer live registers)
+          const float sum = SEL ? relu_wsum_halves(ta, wr) : relu_wsum(ta, wr);
           if constexpr (SEL) {
             tc_fence_before();
             __syncwarp();
@@ -812,14 +840,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (valid) atomicAdd(&ssm->hist[b], 1u);
             const bool keep = valid && b >= thr_w;
             uint32_t cs;
-            if (sel::warp_append(keep, rcnt + sg.r, cs) && keep)
-              cand[(int64_t)sg.r * cap + cs] = sel::pack_cand(sel::rank_key(x), s);
-            if ((++units & 3) == 0) {
+            if (sel::warp_append(keep, scnt, cs) && keep)
+              cand[(int64_t)sg.r * cap + (int64_t)sg.kb * kTileK + cs] =
+                  sel::pack_cand(sel::rank_key(x), s);
+            ++units;
+            if ((units & 7) == 0) {  // this segment's k-th best so far, shared with the row
               const uint32_t bk = kth_bin(ssm->hist, k, lane);
+              if (lane == 0 && bk > thr_w) atomicMax(rthr + sg.r, bk);  // no wait for it
+              thr_w = max(thr_w, bk);
+            }
+            if ((units & 15) == 0) {  // other segments' thresholds, now and then
               uint32_t g = 0;
-              if (lane == 0 && bk > thr_w) g = atomicMax(rthr + sg.r, bk);
-              else if (lane == 0) g = __ldcg(rthr + sg.r);
-              thr_w = max(thr_w, max(bk, __shfl_sync(0xffffffffu, g, 0)));
+              if (lane == 0) g = __ldcg(rthr + sg.r);
+              thr_w = max(thr_w, __shfl_sync(0xffffffffu, g, 0));
             }
           } else {
             if (s < R.max_len) {
@@ -844,20 +877,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!seg_ok) *abort_flag = 1;
         seg_ok = bar_red_and<4, kEpiThreads>(seg_ok);
         if (seg_ok) {
-          const uint32_t seg_tiles = (uint32_t)(sg.ke - sg.kb);
-          const uint32_t row_tiles = (uint32_t)((ri.t + kTileK) / kTileK);
+          // the segment's count and histogram into the row's, then fresh ones
+          uint32_t* const rh = rhist + (int64_t)sg.r * sel::kBins;
+          for (int i = et; i < sel::kBins; i += kEpiThreads) {
+            const uint32_t c = ssm->hist[i];
+            if (c) atomicAdd(rh + i, c);
+            ssm->hist[i] = 0;
+          }
           if (et == 0) {
-            __threadfence();  // this CTA's candidates before its share of the row's tiles
-            *last_flag = atomicAdd(rdone + sg.r, seg_tiles) + seg_tiles == row_tiles ? 1u : 0u;
+            segcnt[(int64_t)sg.r * (cap / kTileK) + sg.kb] = *scnt;
+            *scnt = 0;
           }
-          asm volatile("bar.sync 4, %0;" ::"n"(kEpiThreads) : "memory");
-          if (*last_flag) {  // the row's last segment: select its k best
-            __threadfence();
-            const uint32_t m = __ldcg(rcnt + sg.r);
-            sel::select_list<SelB>(*ssm, cand + (int64_t)sg.r * cap, m, k,
-                                   idx + (int64_t)sg.r * k, ckey, cpos);
-          }
-          for (int i = et; i < sel::kBins; i += kEpiThreads) ssm->hist[i] = 0;
           asm volatile("bar.sync 4, %0;" ::"n"(kEpiThreads) : "memory");
         }
       }
@@ -934,7 +964,8 @@ static dsa_status_t launch_decode(const Rows& R, int32_t row0, int32_t nrows, co
                                   const float* q_scale, const float* w, const void* k_idx,
                                   const float* k_scale, float* scores, int64_t ld, bool fill,
                                   cudaStream_t st, uint64_t* cand = nullptr, int64_t cap = 0,
-                                  uint32_t* rstate = nullptr, int32_t* idx = nullptr, int k = 0) {
+                                  uint32_t* rstate = nullptr, uint32_t* segcnt = nullptr,
+                                  uint32_t* rhist = nullptr, int k = 0) {
   using D = DecCfg<DT, NK, SEL>;
   using C = typename D::C;
   CUtensorMap qmap, kmap;
@@ -948,22 +979,30 @@ static dsa_status_t launch_decode(const Rows& R, int32_t row0, int32_t nrows, co
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
-  if (SEL && cudaMemsetAsync(rstate, 0, sizeof(uint32_t) * 3 * (size_t)nrows, st) != cudaSuccess)
-    return DSA_ERR_CUDA;
   kfn<<<num_sms(), kThreads, D::SMEM, st>>>(qmap, kmap, R, row0, nrows, w, q_scale, k_scale,
-                                            scores, ld, fill ? 1 : 0, cand, cap, rstate, idx, k);
+                                            scores, ld, fill ? 1 : 0, cand, cap, rstate, segcnt,
+                                            rhist, k);
   return launch_status();
 }
 
 bool indexer_select_supported(const Rows& R, int dtype, int H_I, int D_I, int k) {
+  // (the selection kernel takes rows of up to 1024 key tiles)
   return R.mode == DSA_DECODE && indexer_tc_supported(dtype, H_I, D_I) && k >= 1 &&
-         k <= 16384;
+         k <= 16384 && R.max_len <= 1024 * kTileK;
+}
+
+// Workspace of the fused path: the candidate lists ([nrows][cap], cap =
+// max_len rounded up to whole key tiles), then per row its threshold, segment
+// counts and histogram (zeroed before each launch).
+static int64_t select_cap(const Rows& R) { return ((int64_t)R.max_len + kTileK - 1) / kTileK * kTileK; }
+static size_t select_state_words(const Rows& R, int32_t nrows) {
+  return (size_t)nrows * (1 + (size_t)(select_cap(R) / kTileK) + sel::kBins);
 }
 
 size_t indexer_select_workspace(const Rows& R, int32_t nrows) {
   if (nrows <= 0) return 0;
-  const size_t cand = (size_t)nrows * (size_t)R.max_len * sizeof(uint64_t);
-  return (cand + 255) / 256 * 256 + (size_t)nrows * 3 * sizeof(uint32_t);
+  const size_t cand = (size_t)nrows * (size_t)select_cap(R) * sizeof(uint64_t);
+  return (cand + 255) / 256 * 256 + select_state_words(R, nrows) * sizeof(uint32_t);
 }
 
 dsa_status_t launch_indexer_select(const Rows& R, int32_t row0, int32_t nrows, int dtype,
@@ -973,15 +1012,25 @@ dsa_status_t launch_indexer_select(const Rows& R, int32_t row0, int32_t nrows, i
   if (!indexer_select_supported(R, dtype, H_I, D_I, k)) return DSA_ERR_UNSUPPORTED;
   if (nrows <= 0) return DSA_OK;
   if (!ws || ws_bytes < indexer_select_workspace(R, nrows)) return DSA_ERR_WORKSPACE;
+  const int64_t cap = select_cap(R);
   uint64_t* cand = reinterpret_cast<uint64_t*>(ws);
-  const size_t cbytes = ((size_t)nrows * (size_t)R.max_len * sizeof(uint64_t) + 255) / 256 * 256;
+  const size_t cbytes = ((size_t)nrows * (size_t)cap * sizeof(uint64_t) + 255) / 256 * 256;
   uint32_t* rstate = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + cbytes);
-  if (dtype == DSA_BF16)
-    return launch_decode<DSA_BF16, 5, true>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale,
-                                            nullptr, 0, false, st, cand, R.max_len, rstate, idx,
-                                            k);
-  return launch_decode<DSA_E4M3, 11, true>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale,
-                                           nullptr, 0, false, st, cand, R.max_len, rstate, idx, k);
+  uint32_t* segcnt = rstate + nrows;
+  uint32_t* rhist = segcnt + (size_t)nrows * (cap / kTileK);
+  if (cudaMemsetAsync(rstate, 0, select_state_words(R, nrows) * sizeof(uint32_t), st) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  dsa_status_t s =
+      dtype == DSA_BF16
+          ? launch_decode<DSA_BF16, 5, true>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale,
+                                             nullptr, 0, false, st, cand, cap, rstate, segcnt,
+                                             rhist, k)
+          : launch_decode<DSA_E4M3, 12, true>(R, row0, nrows, q_idx, q_scale, w, k_idx, k_scale,
+                                              nullptr, 0, false, st, cand, cap, rstate, segcnt,
+                                              rhist, k);
+  if (s) return s;
+  return launch_select_rows(R, row0, nrows, cand, cap, segcnt, rhist, k, idx, st);
 }
 
 dsa_status_t launch_indexer_tc(const Rows& R, int32_t row0, int32_t nrows, int dtype, int H_I,

@@ -34,6 +34,13 @@ dsa_status_t launch_indexer_select(const Rows& R, int32_t row0, int32_t nrows, i
                                    const float* w, const void* k_idx, const float* k_scale, int k,
                                    int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t st);
 
+// The k best of each row from the fused decode indexer's candidate lists
+// (cand [nrows][cap] in segments, segment counts segcnt [nrows][cap / 128],
+// row histograms rhist [nrows][2048]).
+dsa_status_t launch_select_rows(const Rows& R, int32_t row0, int32_t nrows, const uint64_t* cand,
+                                int64_t cap, const uint32_t* segcnt, const uint32_t* rhist, int k,
+                                int32_t* idx, cudaStream_t st);
+
 // Radix top-k, one CTA per row.
 dsa_status_t launch_topk(const Rows& R, int32_t row0, int32_t nrows, const float* scores,
                          int64_t ld, int k, int32_t* idx, cudaStream_t st);

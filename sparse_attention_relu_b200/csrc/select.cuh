@@ -229,49 +229,61 @@ __device__ __forceinline__ uint64_t pack_cand(uint32_t key, int32_t pos) {
   return ((uint64_t)key << 32) | (uint32_t)pos;
 }
 
-// Radix select of one 11- or 10-bit digit over the entries of `cand[0, m)`
+// Radix select of one 11- or 10-bit digit over the entries get(0 .. m-1)
 // that `member` admits: histogram of digit (v >> shift) & mask in sm.hist,
 // then find_bin for `need`.  The caller folds the digit into its prefix.
-template <class B, class Member, class Value>
-__device__ void radix_level(Smem<B::NW>& sm, const uint64_t* cand, uint32_t m, int shift,
+template <class B, class Get, class Member, class Value>
+__device__ void radix_level(Smem<B::NW>& sm, const Get& get, uint32_t m, int shift,
                             uint32_t width, uint32_t need, Member member, Value value) {
   const int tid = B::tid();
   for (int i = tid; i < kBins; i += B::NT) sm.hist[i] = 0;
   B::sync();
   for (uint32_t i = tid; i < m; i += B::NT) {
-    const uint64_t c = __ldcg(reinterpret_cast<const unsigned long long*>(cand) + i);
+    const uint64_t c = get(i);
     if (member(c)) atomicAdd(&sm.hist[(value(c) >> shift) & ((1u << width) - 1u)], 1u);
   }
   B::sync();
   find_bin<B>(sm, 1 << width, need);
 }
 
-// Exact top-k of a candidate list: the k best of cand[0, m) by key, ties to
-// the lower position, written to out[0, k) in any order (-1 padded when
-// m < k).  The list must hold every score of the row that can be among its k
-// best (then the result is the row's top-k).  cand lives in global memory
-// written earlier by this kernel (read through L2).  ckey / cpos: kCand
-// entries of shared scratch.  All NT threads of B call it.
-template <class B>
-__device__ void select_list(Smem<B::NW>& sm, const uint64_t* cand, uint32_t m, int k,
-                            int32_t* out, uint32_t* ckey, int32_t* cpos) {
+// Exact top-k of a candidate list: the k best of the entries get(0 .. m-1)
+// by key, ties to the lower position, written to out[0, k) in any order (-1
+// padded when m < k).  The list must hold every score of the row that can be
+// among its k best (then the result is the row's top-k).
+// have_hist: sm.hist already holds the bin histogram of the whole row (of
+// which the list holds at least every score in the bins from the k-th best's
+// up), else it is built from the list.  ckey / cpos: kCand entries of shared
+// scratch.  All NT threads of B call it.
+template <class B, class Get>
+__device__ void select_list(Smem<B::NW>& sm, const Get& ld, uint32_t m, int k, int32_t* out,
+                            uint32_t* ckey, int32_t* cpos, bool have_hist = false) {
+  constexpr int RB = 8;  // candidates each thread loads per round (in flight together)
   const int tid = B::tid();
-  auto ld = [&](uint32_t i) {
-    return __ldcg(reinterpret_cast<const unsigned long long*>(cand) + i);
-  };
   if (m <= (uint32_t)k) {
     for (int i = tid; i < k; i += B::NT) out[i] = (uint32_t)i < m ? (int32_t)(uint32_t)ld(i) : -1;
     return;
   }
   // pass 1: the bin b1 that holds the k-th best
-  for (int i = tid; i < kBins; i += B::NT) sm.hist[i] = 0;
+  if (!have_hist) {
+    for (int i = tid; i < kBins; i += B::NT) sm.hist[i] = 0;
+    B::sync();
+    for (uint32_t base = 0; base < m; base += B::NT * RB) {
+      uint64_t c[RB];
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        const uint32_t i = base + tid + B::NT * r;
+        c[r] = i < m ? ld(i) : 0ull;
+      }
+#pragma unroll
+      for (int r = 0; r < RB; ++r)
+        if (base + tid + B::NT * r < m)
+          atomicAdd(&sm.hist[score_bin(key_float((uint32_t)(c[r] >> 32)))], 1u);
+    }
+  }
   if (tid == 0) {
     sm.n_out = 0;
     sm.n_cand = 0;
   }
-  B::sync();
-  for (uint32_t i = tid; i < m; i += B::NT)
-    atomicAdd(&sm.hist[score_bin(key_float((uint32_t)(ld(i) >> 32)))], 1u);
   B::sync();
   find_bin<B>(sm, kBins, (uint32_t)k);
   const uint32_t b1 = sm.sel_bin, above1 = sm.sel_above, in_b1 = sm.hist[b1];
@@ -279,21 +291,32 @@ __device__ void select_list(Smem<B::NW>& sm, const uint64_t* cand, uint32_t m, i
   // pass 2: above b1 -> out; members of b1 -> the buffer when they fit
   const bool collect = in_b1 <= (uint32_t)kCand;
   const uint32_t mbase = (m + 31u) & ~31u;  // whole warps in every trip
-  for (uint32_t base = 0; base < mbase; base += B::NT) {
-    const uint32_t i = base + tid;
-    const uint64_t c = i < m ? ld(i) : 0ull;
-    const uint32_t key = (uint32_t)(c >> 32), b = i < m ? score_bin(key_float(key)) : 0u;
-    const bool gt = i < m && b > b1, eq = collect && i < m && b == b1;
-    uint32_t slot;
-    if (warp_append(gt, &sm.n_out, slot) && gt) out[slot] = (int32_t)(uint32_t)c;
-    if (warp_append(eq, &sm.n_cand, slot) && eq) {
-      ckey[slot] = key;
-      cpos[slot] = (int32_t)(uint32_t)c;
+  for (uint32_t base = 0; base < mbase; base += B::NT * RB) {  // uniform trip count
+    uint64_t cr[RB];
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+      const uint32_t i = base + tid + B::NT * r;
+      cr[r] = i < m ? ld(i) : 0ull;
+    }
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+      const uint32_t i = base + tid + B::NT * r;
+      const uint64_t c = cr[r];
+      const uint32_t key = (uint32_t)(c >> 32), b = i < m ? score_bin(key_float(key)) : 0u;
+      const bool gt = i < m && b > b1, eq = collect && i < m && b == b1;
+      uint32_t slot;
+      if (warp_append(gt, &sm.n_out, slot) && gt && slot < (uint32_t)k)
+        out[slot] = (int32_t)(uint32_t)c;
+      if (warp_append(eq, &sm.n_cand, slot) && eq && slot < (uint32_t)kCand) {
+        ckey[slot] = key;
+        cpos[slot] = (int32_t)(uint32_t)c;
+      }
     }
   }
   B::sync();
   if (collect) {
-    rank_candidates<B>(sm, ckey, cpos, (int)in_b1, (uint32_t)k - above1, out + above1);
+    const uint32_t nc = sm.n_cand < in_b1 ? sm.n_cand : in_b1;  // equal for a valid list
+    rank_candidates<B>(sm, ckey, cpos, (int)nc, (uint32_t)k - above1, out + above1);
     return;
   }
   // b1 overflows the buffer: radix levels over its members' keys find the
@@ -309,7 +332,7 @@ __device__ void select_list(Smem<B::NW>& sm, const uint64_t* cand, uint32_t m, i
   for (int lvl = 0; lvl < 3; ++lvl) {
     const int hi = dshift(lvl) + (int)dwidth(lvl);
     const uint32_t pre = prefix;
-    radix_level<B>(sm, cand, m, dshift(lvl), dwidth(lvl), (uint32_t)k - c_gt,
+    radix_level<B>(sm, ld, m, dshift(lvl), dwidth(lvl), (uint32_t)k - c_gt,
                    [&](uint64_t c) { return in_b1f(c) && (hi >= 32 || (keyf(c) >> hi) == pre); },
                    keyf);
     prefix = (prefix << dwidth(lvl)) | sm.sel_bin;
@@ -327,7 +350,7 @@ __device__ void select_list(Smem<B::NW>& sm, const uint64_t* cand, uint32_t m, i
   for (int lvl = 0; lvl < 3; ++lvl) {
     const int hi = dshift(lvl) + (int)dwidth(lvl);
     const uint32_t pre = pprefix;
-    radix_level<B>(sm, cand, m, dshift(lvl), dwidth(lvl), need_eq - p_gt,
+    radix_level<B>(sm, ld, m, dshift(lvl), dwidth(lvl), need_eq - p_gt,
                    [&](uint64_t c) { return eqf(c) && (hi >= 32 || (rpos(c) >> hi) == pre); },
                    rpos);
     pprefix = (pprefix << dwidth(lvl)) | sm.sel_bin;

@@ -513,7 +513,90 @@ __global__ void __cluster_dims__(P, 1, 1) __launch_bounds__(kThreads, 2)
   }
 }
 
+// The rows' k best from the candidate lists of the fused decode indexer
+// (indexer_decode_kernel with SEL): one CTA per row.  A row's list is in
+// segments: the segment that starts at key tile j holds segcnt[j] entries at
+// cand[j * 128 ...].  The row's histogram, built by the indexer over all its
+// scores, fixes the bin b1 of the k-th best; the segments hold every score of
+// b1 and above, from which the k best are written as select_list does.  Rows
+// with n <= k candidates take 0 .. n-1.
+constexpr int kMaxSeg = 1024;  // segments a row can have (one per key tile at most)
+__global__ void __launch_bounds__(kThreads, 1)
+    select_rows_kernel(Rows R, int32_t row0, const uint64_t* __restrict__ cand, int64_t cap,
+                       const uint32_t* __restrict__ segcnt, const uint32_t* __restrict__ rhist,
+                       int k, int32_t* __restrict__ idx) {
+  __shared__ uint32_t ckey[kCand];
+  __shared__ int32_t cpos[kCand];
+  __shared__ Smem sm;
+  __shared__ uint32_t seg_first[kMaxSeg];  // entry offset of the segment's list in the row
+  __shared__ uint32_t seg_pre[kMaxSeg + 1];  // candidates before the segment
+  __shared__ int nseg;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int32_t r = blockIdx.x;
+  const RowInfo ri = row_info(R, row0 + r);
+  const int n = ri.t + 1;
+  int32_t* out = idx + (int64_t)r * k;
+  if (n <= k) {
+    for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  // the row's segments, in tile order (a warp-wide scan of the tile counts)
+  const int ntile = (int)((n + 127) / 128);
+  const uint32_t* sc = segcnt + (int64_t)r * (cap / 128);
+  if (tid < 32) {
+    uint32_t total = 0;
+    int ns = 0;
+    for (int j0 = 0; j0 < ntile && j0 < kMaxSeg; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t c = j < ntile ? __ldcg(sc + j) : 0u;
+      const uint32_t nz = __ballot_sync(0xffffffffu, c != 0);
+      uint32_t incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (c) {
+        const int slot = ns + __popc(nz & ((1u << lane) - 1u));
+        seg_first[slot] = (uint32_t)j * 128u;
+        seg_pre[slot] = total + incl - c;
+      }
+      total += __shfl_sync(0xffffffffu, incl, 31);
+      ns += __popc(nz);
+    }
+    if (lane == 0) {
+      seg_pre[ns] = total;
+      nseg = ns;
+    }
+  }
+  const uint32_t* h = rhist + (int64_t)r * kBins;
+  for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = __ldcg(h + i);
+  __syncthreads();
+  const int ns = nseg;
+  const uint32_t m = seg_pre[ns];
+  const unsigned long long* row = reinterpret_cast<const unsigned long long*>(cand + (int64_t)r * cap);
+  // entry i of the row's list: its segment by binary search over the prefix counts
+  auto get = [&](uint32_t i) -> uint64_t {
+    int lo = 0, hi = ns - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (seg_pre[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    return __ldcg(row + seg_first[lo] + (i - seg_pre[lo]));
+  };
+  sel::select_list<B512>(sm, get, m, k, out, ckey, cpos, true);
+}
+
 }  // namespace
+
+dsa_status_t launch_select_rows(const Rows& R, int32_t row0, int32_t nrows, const uint64_t* cand,
+                                int64_t cap, const uint32_t* segcnt, const uint32_t* rhist, int k,
+                                int32_t* idx, cudaStream_t st) {
+  if (nrows <= 0) return DSA_OK;
+  if (cap / 128 > kMaxSeg || cap % 128) return DSA_ERR_UNSUPPORTED;
+  select_rows_kernel<<<nrows, kThreads, 0, st>>>(R, row0, cand, cap, segcnt, rhist, k, idx);
+  return launch_status();
+}
 
 dsa_status_t launch_topk(const Rows& R, int32_t row0, int32_t nrows, const float* scores,
                          int64_t ld, int k, int32_t* idx, cudaStream_t st) {

@@ -34,7 +34,7 @@ def _timed(fn):
     return e0.elapsed_time(e1)
 
 
-def attn(case: str, reps: int, T: int, k: int = 2048):
+def attn(case: str, reps: int, T: int, k: int = 2048, kv_dtype: str = "bf16"):
     dev = "cuda"
     torch.manual_seed(0)
     if case == "prefill":
@@ -59,21 +59,34 @@ def attn(case: str, reps: int, T: int, k: int = 2048):
         j = torch.arange(k, device=dev)[None, :]
         idx = (j * 7 + 131 * torch.arange(B, device=dev)[:, None]) % L
     idx = idx.to(torch.int32).contiguous()
-    kv = (torch.randn(n_k, 576, device=dev) / 24).to(torch.bfloat16)
+    kv32 = torch.randn(n_k, 576, device=dev) / 24
+    kv_scale = None
+    if kv_dtype == "e4m3":
+        import workloads
+
+        kv, kv_scale = workloads.quantize_e4m3_per_token(kv32)
+    else:
+        kv = kv32.to(torch.bfloat16)
+    del kv32
     q = (torch.randn(n_q, 128, 576, device=dev) / 24).to(torch.bfloat16)
     out = torch.empty(n_q, 128, 512, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(n_q, 128, dtype=torch.float32, device=dev)
     nws = dsa.dsa_sparse_mla_attn_workspace_size(lay, k, 128, 576, 512)
     ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
-    run = lambda: dsa.dsa_sparse_mla_attn(lay, q, kv, idx, k, 512, 1 / 24, out, lse, ws)
+    if kv_scale is None:
+        run = lambda: dsa.dsa_sparse_mla_attn(lay, q, kv, idx, k, 512, 1 / 24, out, lse, ws)
+    else:
+        run = lambda: dsa.dsa_sparse_mla_attn_e4m3(lay, q, kv, kv_scale, idx, k, 512, 1 / 24, out,
+                                                   lse, ws)
     for _ in range(reps):
         run()
     torch.cuda.synchronize()
     assert dsa.dsa_device_status() == 0
     ms = _timed(run)
     sel = (idx >= 0).sum().item()
-    print(f"attn/{case}: rows={n_q} selected={sel} ms={ms:.3f} "
-          f"TFLOP/s={sel * 278528 / ms / 1e9:.1f} gather GB/s={sel * 1152 / ms / 1e6:.1f}")
+    row_bytes = 1152 if kv_scale is None else 580
+    print(f"attn/{case} ({kv_dtype} cache): rows={n_q} selected={sel} ms={ms:.3f} "
+          f"TFLOP/s={sel * 278528 / ms / 1e9:.1f} gather GB/s={sel * row_bytes / ms / 1e6:.1f}")
 
 
 def indexer_topk(stage: str, reps: int, T: int, k: int = 2048):
@@ -107,9 +120,10 @@ def main():
     ap.add_argument("--case", choices=["prefill", "decode"], default="prefill")
     ap.add_argument("--reps", type=int, default=4)
     ap.add_argument("--tokens", type=int, default=None)
+    ap.add_argument("--kv", choices=["bf16", "e4m3"], default="bf16", help="MLA cache storage")
     a = ap.parse_args()
     if a.stage == "attn":
-        attn(a.case, a.reps, a.tokens or 4096)
+        attn(a.case, a.reps, a.tokens or 4096, kv_dtype=a.kv)
     else:
         indexer_topk(a.stage, a.reps, a.tokens or 16384)
 
