@@ -101,7 +101,7 @@ def algorithmic_work(wl):
 
 # decode end to end: rows per slab of dsa_forward_host (the copies of one slab
 # overlap the kernels of another)
-DECODE_SLAB_ROWS = 16
+DECODE_SLAB_ROWS = 32
 
 SPIN_CYCLES = 1_000_000  # about 0.5 ms at 1.9-2 GHz, longer than the host takes to queue a step
 
@@ -189,7 +189,8 @@ def describe(cfg):
     return d
 
 
-def run_device(cid, steps, warmup, rank, world, do_e2e=True, index_reuse=1, kv_dtype="bf16"):
+def run_device(cid, steps, warmup, rank, world, do_e2e=True, index_reuse=1, kv_dtype="bf16",
+               decode_slab_rows=None):
     import sparse_attention_relu_b200 as dsa
 
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -254,7 +255,7 @@ def run_device(cid, steps, warmup, rank, world, do_e2e=True, index_reuse=1, kv_d
 
     e2e = None
     if do_e2e:
-        e2e = run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream)
+        e2e = run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream, decode_slab_rows)
     reuse = None
     if index_reuse > 1:
         reuse = run_index_reuse(dsa, wl, lay, args, out, lse, ws, flush, stream, steps, warmup,
@@ -328,7 +329,7 @@ def run_index_reuse(dsa, wl, lay, args, out, lse, ws, flush, stream, steps, warm
             "later_layer_ms": (ms - ms1) / (layers - 1)}
 
 
-def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
+def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream, decode_slab_rows=None):
     """Same metric through the public API with host buffers: every step copies
     the step's inputs from pinned host memory and reads the result back.
 
@@ -379,7 +380,7 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
     # side); decode rows run in slabs of DECODE_SLAB_ROWS so that its copies
     # overlap too
     use_host = True
-    slab_cap = DECODE_SLAB_ROWS if c.mode == "decode" else 0
+    slab_cap = (decode_slab_rows or DECODE_SLAB_ROWS) if c.mode == "decode" else 0
     if use_host:
         hargs = dsa.forward_args(q_idx=host["q_idx"], q_scale=host.get("q_scale"), w=host["w"],
                                  k_idx=host.get("k_idx"), k_scale=host.get("k_scale"),
@@ -428,18 +429,20 @@ def run_e2e(dsa, wl, lay, c, dev, steps, d, ws, stream):
 KERNEL_SOURCES = {"indexer": "indexer_tc.cu", "topk": "topk.cu", "sparse_mla_attn": "attn_tc.cu"}
 
 
-def measured_traffic(kernel, cid):
+def measured_traffic(kernel, cfg):
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
-    `kernel` on workload `cid`, from the ncu capture recorded in
-    profiles/dram_traffic.json -- or None when there is none, or when the
-    kernel's source has changed since (the record keeps its SHA-256)."""
+    `kernel` on workload `cfg` (its id, and its cache type when not bf16), from
+    the ncu capture recorded in profiles/dram_traffic.json -- or None when
+    there is none, or when the kernel's source has changed since (the record
+    keeps its SHA-256)."""
     import hashlib
 
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
         return None
+    key = f"{kernel}/{cfg.cid}" + ("" if cfg.kv_dtype == "bf16" else f"/{cfg.kv_dtype}")
     with open(path) as f:
-        rec = json.load(f).get(f"{kernel}/{cid}")
+        rec = json.load(f).get(key)
     if not rec:
         return None
     src = os.path.join(ROOT, "sparse_attention_relu_b200", "csrc", KERNEL_SOURCES[kernel])
@@ -490,7 +493,7 @@ def roofline(wl, stage_ms, peaks):
     shares = {names[k]: round(v / sum(tot.values()), 4) for k, v in tot.items()}
     return {"kernel": names[kind], "bound": bound, "achieved": round(achieved, 2),
             "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
-            "traffic": measured_traffic(names[kind], c.cid),
+            "traffic": measured_traffic(names[kind], c),
             "peak_source": peaks["source"] + (" (x2 nominal fp8/bf16 ratio)" if
                                              unit == "TFLOP/s" and kind == 0 and
                                              c.idx_dtype == "e4m3" else ""),
@@ -608,6 +611,9 @@ def main():
     ap.add_argument("--kv-dtype", default="bf16", choices=["bf16", "e4m3"],
                     help="storage of the MLA cache: bf16, or FP8 e4m3 codes with per-token "
                          "scales (dsa_sparse_mla_attn_e4m3)")
+    ap.add_argument("--decode-slab-rows", type=int, default=None,
+                    help=f"decode end to end: rows per slab of dsa_forward_host "
+                         f"(default {DECODE_SLAB_ROWS})")
     ap.add_argument("--index-reuse", type=int, default=1,
                     help="L > 1 adds an `index_reuse` object: one indexer serving L attention "
                          "layers (IndexCache), tokens/s of the L-layer step")
@@ -633,12 +639,14 @@ def main():
                                              device_id=torch.device("cuda", local))
     peaks = load_peaks()
     wl, ms, stage_ms, launches, clocks, e2e, reuse = run_device(
-        cid, a.steps, a.warmup, rank, world, not a.no_e2e, a.index_reuse, a.kv_dtype)
+        cid, a.steps, a.warmup, rank, world, not a.no_e2e, a.index_reuse, a.kv_dtype,
+        a.decode_slab_rows)
     dec = None
     if a.decode_workload != "none":
         dcid = WORKLOADS[a.decode_workload]
         dwl, dms, dstage, dlaunch, _, de2e, dreuse = run_device(
-            dcid, a.steps, a.warmup, rank, world, not a.no_e2e, a.index_reuse, a.kv_dtype)
+            dcid, a.steps, a.warmup, rank, world, not a.no_e2e, a.index_reuse, a.kv_dtype,
+            a.decode_slab_rows)
         dec = (dwl, dms, dstage, dlaunch, de2e, dreuse)
 
     ms = max_over_ranks(ms, world, "cuda")

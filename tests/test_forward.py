@@ -63,9 +63,14 @@ def test_sampled_rows_cover_slab_boundaries(cid):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("cid", [1, 2, 3, 4, 5, 6])
-def test_forward_matches_oracle(cid):
-    wl = workloads.generate(cid)
+@pytest.mark.parametrize("cid,kv_dtype", [(1, "bf16"), (2, "bf16"), (3, "bf16"), (4, "bf16"),
+                                          (5, "bf16"), (6, "bf16"), (2, "e4m3"), (3, "e4m3"),
+                                          (4, "e4m3"), (5, "e4m3")])
+def test_forward_matches_oracle(cid, kv_dtype):
+    """kv_dtype e4m3: the same workload with an FP8 MLA cache (per-token scales)."""
+    cfg = workloads.config(cid)
+    cfg.kv_dtype = kv_dtype
+    wl = workloads.generate(cfg)
     dev = Dev(wl)
     out, lse, idx = dev.forward()
     assert dev.status() == dsa.DSA_OK
