@@ -27,15 +27,21 @@
 //   atoms), two stages of 64 gathered cache rows (nine atoms of 64 dims,
 //   K-major for QK, MN-major for PV), and the tile's probabilities P (bf16,
 //   K-major) for PV.
-// The gather: 224 producer threads fetch the QK-only atoms of each tile and
-// the 256 softmax threads, idle while the tensor cores work on the next
-// tile, fetch this CTA's value atoms, all with 16-byte cp.async, eight lanes
-// per 128-byte segment, straight into the swizzled
-// layout the MMA reads (an empty slot -1 is zero-filled).  Measured on B200
-// (scattered rows, L2-resident source): cp.async sustains about 16 B/cycle
-// per SM from 2 producer warps, 30 from 4 and 40 from 16 -- a warp keeps a
-// bounded number of bytes in flight -- while one thread issuing TMA
-// tile::gather4 (4 rows per instruction) manages about 4.
+// The query row arrives by TMA (nine 16 KB boxes, one per 64-dim atom of
+// all heads): dims 384..575 straight into their operand atoms, dims 0..383
+// staged in the not yet used gather stages, from which the softmax threads
+// move them into TMEM.  (Loaded by each softmax thread from its own head's
+// row, the query took about 20K cycles of a CTA's start.)
+// The gather: 224 producer threads publish each tile's indices and fetch its
+// rows with 16-byte cp.async, eight lanes per 128-byte segment, straight into
+// the swizzled layout the MMA reads (an empty slot -1 is zero-filled).
+// Measured on B200 (scattered 128-byte rows, L2-resident source, 208 KB of
+// shared memory per CTA): cp.async from 7 warps sustains 20 B/cycle per SM,
+// from 15 warps 27; TMA tile::gather4 from 8 issuing threads 28, and
+// cp.async and gather4 issued together stay at 28 (one limit for both).
+// Inside this kernel, gather4 from lane 0 of the 7 producer warps was slower
+// than cp.async (6.2 against 5.0 ms on 4096 prefill rows): one thread issues
+// a gather4 only about every 120 cycles.
 //
 // Warp roles (512 threads per CTA):
 //   warps 0-6   gather producer (indices -> shared memory, cp.async rows)
@@ -51,6 +57,8 @@
 // normalised partial output and its log-sum-exp, merged by
 // attn_combine_kernel.
 #include <cudaTypedefs.h>
+
+#include <cstdint>
 
 #include "kernels.cuh"
 #include "sm100.cuh"
@@ -94,7 +102,7 @@ constexpr int OFF_MASK = OFF_IDX + kIdxRing * kNT * 4;   // [ring][2] uint32 val
 constexpr int OFF_HMAX = OFF_MASK + kIdxRing * 2 * 4;    // [2 tiles][2 warpgroups][128] float
 constexpr int OFF_KSC = OFF_HMAX + 2 * 2 * kH * 4;       // [ring][64] fp32 cache scales (e4m3)
 constexpr int OFF_BAR = OFF_KSC + kIdxRing * kNT * 4;
-constexpr int kNumBars = 22;
+constexpr int kNumBars = 23;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 // The dynamic window starts 1024-aligned (right after the driver's reserved
 // kilobyte, with no static shared memory); the kernel checks it.
@@ -127,9 +135,10 @@ enum {
   B_PFULL = 11,   // P stored (every softmax thread)
   B_PVDONE = 12,  // PV retired
   B_DRAIN = 13,
-  B_IDX = 14      // [kIdxRing] the tile's indices, mask and scales are in the ring (producers)
+  B_IDX = 14,     // [kIdxRing] the tile's indices, mask and scales are in the ring (producers)
+  B_QLOAD = 22    // the query row landed (TMA transaction bytes)
 };
-static_assert(B_IDX + kIdxRing <= kNumBars, "barrier count");
+static_assert(B_IDX + kIdxRing <= B_QLOAD && B_QLOAD < kNumBars, "barrier count");
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
@@ -259,9 +268,11 @@ inline Split plan_split(int32_t nrows, int k) {
 // same swizzled bf16 operand, exactly converted; the MMAs are the bf16 ones.
 // The token's scale multiplies its score column and its probability in the
 // PV operand (P' = p * scale); the softmax denominator sums p.
+// qmap: the queries as a [n_q * 128, 576] bf16 map, 64 x 128 boxes, 128-byte
+// swizzle (one box = one K-major operand atom of all heads).
 template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const uint16_t* __restrict__ q, const void* __restrict__ kv,
+    attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const void* __restrict__ kv,
                    const float* __restrict__ kv_scale, Rows R,
                    int32_t row0, const int32_t* __restrict__ idx, int k, float scale2, Split sp,
                    uint16_t* __restrict__ out, float* __restrict__ lse,
@@ -307,8 +318,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_PFULL), kSoftmaxThreads);
     mbar_init(bar(B_PVDONE), 1);
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_QLOAD), 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // The query row by TMA, nine atoms of 128 heads x 64 dims: dims 384..575
+    // straight into their operand atoms, dims 0..383 staged in the gather
+    // stages (unused until the softmax threads have moved them into TMEM).
+    tma_prefetch(&qmap);
+    mbar_expect_tx(bar(B_QLOAD), (uint32_t)(kH * kDK * 2));
+    for (int a = 0; a < kAtoms; ++a) {
+      const uint32_t dst = a < kQTmemDims / 64 ? sb + OFF_C + a * kQAtomBytes
+                                               : sb + OFF_Q + (a - kQTmemDims / 64) * kQAtomBytes;
+      tma_load_2d(dst, &qmap, 64 * a, r * kH, bar(B_QLOAD));
+    }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(sb + OFF_MISC, 512);
@@ -414,7 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int n = 0; n < ntiles; ++n) {
         const int st = n % kStages;
         const uint32_t par = ((n / kStages) & 1) ^ 1;
-        bool ok = mbar_wait(bar(B_AEMPTY + st), par, R.status) &&
+        // (the first tile also waits until the staged query has left the stages)
+        bool ok = (n > 0 || mbar_wait(bar(B_QREADY), 0, R.status)) &&
+                  mbar_wait(bar(B_AEMPTY + st), par, R.status) &&
                   mbar_wait(bar(B_VEMPTY + st), par, R.status) && !*abort_flag;
         if (!bar_and<2, kProducers>(ok)) {
           *abort_flag = 1;
@@ -449,8 +473,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int n = 0; n < ntiles; ++n) {
         const int st = n % kStages, ring = n % kIdxRing;
         const uint32_t par = ((n / kStages) & 1) ^ 1;
-        // group A of the stage is free once QK(n-2) read it
-        bool ok = mbar_wait(bar(B_AEMPTY + st), par, R.status) && !*abort_flag;
+        // group A of the stage is free once QK(n-2) read it (and, for the
+        // first tile, once the staged query has left the stages)
+        bool ok = (n > 0 || mbar_wait(bar(B_QREADY), 0, R.status)) &&
+                  mbar_wait(bar(B_AEMPTY + st), par, R.status) && !*abort_flag;
         if (!bar_and<2, kProducers>(ok)) {
           *abort_flag = 1;
           break;
@@ -596,45 +622,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint16_t* qrow = q + ((int64_t)r * kH + h) * kDK;
     {
-      // query dims 0..383 -> TMEM columns 0..191 (warpgroup wg: 192 dims)
+      // query dims 0..383 -> TMEM columns 0..191 (warpgroup wg: 192 dims),
+      // read from the atoms the TMA staged in the gather stages
+      const bool q_ok = mbar_wait(bar(B_QLOAD), 0, R.status);
+      if (!q_ok) *abort_flag = 1;
+      if (q_ok) {
 #pragma unroll
-      for (int part = 0; part < 4; ++part) {  // 4 x 48 dims = 4 x 24 columns
-        const uint4* qs = reinterpret_cast<const uint4*>(qrow + 192 * wg + 48 * part);
-        uint32_t w24[24];
+        for (int part = 0; part < 4; ++part) {  // 4 x 48 dims = 4 x 24 columns
+          uint32_t w24[24];
 #pragma unroll
-        for (int v = 0; v < 6; ++v) {
-          const uint4 x = __ldg(qs + v);
-          w24[4 * v] = x.x;
-          w24[4 * v + 1] = x.y;
-          w24[4 * v + 2] = x.z;
-          w24[4 * v + 3] = x.w;
+          for (int v = 0; v < 6; ++v) {
+            const int d = 192 * wg + 48 * part + 8 * v, a = d >> 6, ch = (d >> 3) & 7;
+            const uint4 x = *reinterpret_cast<const uint4*>(
+                smem + OFF_C + a * kQAtomBytes + h * 128 + ((ch ^ (h & 7)) << 4));
+            w24[4 * v] = x.x;
+            w24[4 * v + 1] = x.y;
+            w24[4 * v + 2] = x.z;
+            w24[4 * v + 3] = x.w;
+          }
+          const uint32_t ta = tmem + lane_off + TM_Q + 96 * wg + 24 * part;
+          uint32_t a8[8], b8[8], c8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            a8[e] = w24[e];
+            b8[e] = w24[8 + e];
+            c8[e] = w24[16 + e];
+          }
+          tmem_st8(ta, a8);
+          tmem_st8(ta + 8, b8);
+          tmem_st8(ta + 16, c8);
         }
-        const uint32_t ta = tmem + lane_off + TM_Q + 96 * wg + 24 * part;
-        uint32_t a8[8], b8[8], c8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          a8[e] = w24[e];
-          b8[e] = w24[8 + e];
-          c8[e] = w24[16 + e];
-        }
-        tmem_st8(ta, a8);
-        tmem_st8(ta + 8, b8);
-        tmem_st8(ta + 16, c8);
       }
-      // query dims 384..575 -> three K-major atoms in shared memory (row h;
-      // warpgroup wg stores 16-byte chunks 12wg .. 12wg+11 of the 24)
-#pragma unroll
-      for (int c = 0; c < 12; ++c) {
-        const int chunk = 12 * wg + c, a = chunk >> 3, ch = chunk & 7;
-        const uint4 x = __ldg(reinterpret_cast<const uint4*>(qrow + kQTmemDims + 8 * chunk));
-        *reinterpret_cast<uint4*>(smem + OFF_Q + a * kQAtomBytes + h * 128 +
-                                  ((ch ^ (h & 7)) << 4)) = x;
-      }
-      fence_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(B_QREADY));
+      mbar_arrive(bar(B_QREADY));  // the staged atoms are read: the stages are free
     }
     // row h of P: this warpgroup's 32 rows are 16-byte chunks 4wg .. 4wg+3
     uint8_t* const prow = smem + OFF_P + h * 128;
@@ -775,6 +796,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // the query load has landed before the CTA may exit (it has, unless a wait
+  // above gave up)
+  if (tid == 0) mbar_wait(bar(B_QLOAD), 0, R.status);
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
@@ -842,12 +866,18 @@ dsa_status_t launch_attn_tc(const Rows& R, int32_t row0, int32_t nrows, const ui
     part_o = reinterpret_cast<float*>(ws);
     part_lse = part_o + (size_t)nrows * sp.nsplit * kH * kDV;
   }
+  // the queries as [n_q * 128, 576] (row coordinates r * 128 are 32-bit)
+  if ((int64_t)R.n_q * kH >= INT32_MAX) return DSA_ERR_INVALID_ARGUMENT;
+  CUtensorMap qmap;
+  if (!make_tmap_2d(&qmap, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, (uint64_t)R.n_q * kH, 64,
+                    kH))
+    return DSA_ERR_CUDA;
   auto kfn = kv_scale ? attn_tc_kernel<true> : attn_tc_kernel<false>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
     return DSA_ERR_CUDA;
   const dim3 grid(2 * nrows * sp.nsplit);
-  kfn<<<grid, kThreads, kSmem, st>>>(q, kv, kv_scale, R, row0, idx, k, sm_scale * kLog2e, sp, out,
-                                     lse, part_o, part_lse);
+  kfn<<<grid, kThreads, kSmem, st>>>(qmap, kv, kv_scale, R, row0, idx, k, sm_scale * kLog2e, sp,
+                                     out, lse, part_o, part_lse);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (sp.nsplit > 1) {
     attn_combine_kernel<<<dim3(nrows, kH), 128, 0, st>>>(row0, sp.nsplit, part_o, part_lse, out,
