@@ -33,8 +33,9 @@
 // move them into TMEM.  (Loaded by each softmax thread from its own head's
 // row, the query took about 20K cycles of a CTA's start.)
 // The gather: 224 producer threads publish each tile's indices and fetch its
-// rows with 16-byte cp.async, eight lanes per 128-byte segment, straight into
-// the swizzled layout the MMA reads (an empty slot -1 is zero-filled).
+// QK-only atoms, the 256 softmax threads its value atoms (bf16 cache), all
+// with 16-byte cp.async, eight lanes per 128-byte segment, straight into the
+// swizzled layout the MMA reads (an empty slot -1 is zero-filled).
 // Measured on B200 (scattered 128-byte rows, L2-resident source, 208 KB of
 // shared memory per CTA): cp.async from 7 warps sustains 20 B/cycle per SM,
 // from 15 warps 27; TMA tile::gather4 from 8 issuing threads 28, and
@@ -44,7 +45,8 @@
 // a gather4 only about every 120 cycles.
 //
 // Warp roles (512 threads per CTA):
-//   warps 0-6   gather producer (indices -> shared memory, cp.async rows)
+//   warps 0-6   gather producer (indices -> shared memory, cp.async of the
+//               QK-only atoms; of every atom for an e4m3 cache, via registers)
 //   warp 7      TMEM allocator and MMA issuer (one thread, issues whichever of
 //               QK(next tile) and PV(oldest tile with P ready) can go)
 //   warps 8-15  softmax, two warpgroups: a thread owns one head (its TMEM
@@ -52,7 +54,8 @@
 //               log2 domain with a lazy rescale (the reference max moves only
 //               when a new score exceeds it by more than 2^8); P to shared
 //               memory as bf16; the denominator sums the fp32 probabilities;
-//               final normalisation and store of this CTA's output columns.
+//               cp.async of the next tile's value atoms (bf16 cache); final
+//               normalisation and store of this CTA's output columns.
 // Decode rows are split over several CTA pairs; each split writes a
 // normalised partial output and its log-sum-exp, merged by
 // attn_combine_kernel.
@@ -308,7 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kStages; ++i) {
       // per producer: an arrive after the index store and a cp.async arrive
       mbar_init(bar(B_AFULL + i), 2 * kProducers);
-      mbar_init(bar(B_VFULL + i), kProducers);  // a cp.async arrive (or arrive) per producer
+      // group V: a cp.async arrive per softmax thread (bf16) or an arrive per producer (e4m3)
+      mbar_init(bar(B_VFULL + i), FP8 ? kProducers : kSoftmaxThreads);
       mbar_init(bar(B_AEMPTY + i), 1);
       mbar_init(bar(B_VEMPTY + i), 1);
     }
@@ -341,9 +345,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  const char* kvb = reinterpret_cast<const char*>(kv) + ri.kbase * kRowBytes;
+  // bf16 cache: issues 16-byte chunk i of atom group A or V (eight lanes per
+  // 128-byte segment of a row, a warp four consecutive segments) of the tile
+  // whose indices are in ring slot `ring` into stage st.
+  auto issue = [&](int st, int ring, int i, bool group_a) {
+    const int ch = i & 7, seg = i >> 3;
+    int row, atom;
+    if (group_a) {  // the five atoms only QK reads
+      row = seg / kAtomsA;
+      const int ai = seg - row * kAtomsA;
+      atom = ai < 4 ? 4 * (half ^ 1) + ai : 8;
+    } else {  // this CTA's value columns
+      row = seg >> 2;
+      atom = 4 * half + (seg & 3);
+    }
+    const int32_t s = sidx[ring * kNT + row];
+    const char* src = s >= 0 ? kvb + (int64_t)s * kRowBytes + atom * 128 + ch * 16
+                             : reinterpret_cast<const char*>(kv);
+    const uint32_t nbytes = s >= 0 ? 16u : 0u;  // 0: zero-fill
+    const uint32_t dst = sb + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128 +
+                         ((uint32_t)(ch ^ (row & 7)) << 4);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(nbytes)
+                 : "memory");
+  };
+
   if (warp < kMmaWarp) {
     // ------------------------------------------------------------ gather producer
-    const char* kvb = reinterpret_cast<const char*>(kv) + ri.kbase * kRowBytes;
     auto load_idx = [&](int n) -> int32_t {
       const int slot = slot_lo + n * kNT + tid;
       int32_t s = slot < slot_hi ? __ldg(idx + (int64_t)rloc * k + slot) : -1;
@@ -361,29 +389,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Threads 0..63 own the index (and scale) of tile row tid.
     int32_t pre = (tid < kNT && ntiles > 0) ? load_idx(0) : -1;
     float pre_sc = load_scale(pre);
-    // Issues 16-byte chunk i of group G (eight lanes per 128-byte segment of
-    // a row, a warp four consecutive segments) of tile n into stage st.
-    auto issue = [&](int st, int ring, int i, bool group_a) {
-      const int ch = i & 7, seg = i >> 3;
-      int row, atom;
-      if (group_a) {  // the five atoms only QK reads
-        row = seg / kAtomsA;
-        const int ai = seg - row * kAtomsA;
-        atom = ai < 4 ? 4 * (half ^ 1) + ai : 8;
-      } else {  // this CTA's value columns
-        row = seg >> 2;
-        atom = 4 * half + (seg & 3);
-      }
-      const int32_t s = sidx[ring * kNT + row];
-      const char* src = s >= 0 ? kvb + (int64_t)s * kRowBytes + atom * 128 + ch * 16
-                               : reinterpret_cast<const char*>(kv);
-      const uint32_t nbytes = s >= 0 ? 16u : 0u;  // 0: zero-fill
-      const uint32_t dst = sb + OFF_C + st * kCBytes + atom * kAtomBytes + row * 128 +
-                           ((uint32_t)(ch ^ (row & 7)) << 4);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                   "r"(nbytes)
-                   : "memory");
-    };
     // Publishes the indices (and mask and scales) of tile n into ring slot
     // n % kIdxRing (threads 0..63 hold them in pre / pre_sc), then loads tile
     // n+1's into pre / pre_sc.
@@ -488,20 +493,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
                          bar(B_AFULL + st))
                      : "memory");
-        // group V of the stage (this CTA's value columns) is free once PV(n-2)
-        // read it; the producers fetch it too, so that the softmax threads
-        // never wait for a PV to retire
-        ok = mbar_wait(bar(B_VEMPTY + st), par, R.status) && !*abort_flag;
-        if (!bar_and<2, kProducers>(ok)) {
-          *abort_flag = 1;
-          break;
-        }
-#pragma unroll
-        for (int j = 0; j < (kChunksV + kProducers - 1) / kProducers; ++j)
-          if (tid + kProducers * j < kChunksV) issue(st, ring, tid + kProducers * j, false);
-        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
-                         bar(B_VFULL + st))
-                     : "memory");
+        // (group V, this CTA's value columns, is fetched by the softmax
+        // threads once PV(n-2) has released it)
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
@@ -509,12 +502,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(bar(B_QREADY), 0, R.status);
-      // Three kinds of work, issued as soon as they can go (PV first):
+      // Three kinds of work, issued as soon as they can go (bf16 cache: QK-B
+      // first, then PV, then QK-A):
       //   QK-A(n): the 20 K steps over group A (rows landed, score tile free)
       //   QK-B(n): the 16 K steps over group V, then S(n) is complete
       //   PV(n):   P(n) stored
-      // Splitting QK lets PV(n-1) slip in between QK-A(n) and QK-B(n), and
-      // group A of a stage is released as soon as its QK steps retire.
+      // Splitting QK lets PV(n-1) slip in between QK-A(n) and QK-B(n) when
+      // group V of tile n is late, and group A of a stage is released as soon
+      // as its QK steps retire.  With QK-B(n) ahead of PV(n-1) when both can
+      // go, S(n) completes earlier and PV(n-1) runs while the softmax threads
+      // read it (measured 4.28 against 4.60 ms on 4096 prefill rows, together
+      // with the softmax-side fetch of group V).
       // Polling uses the non-blocking test: try_wait may suspend the thread
       // while another of the three could already go.
       int na = 0, nb = 0, np = 0;
@@ -543,23 +541,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         bool progressed = false;
-        if (np < nb && mbar_test(bar(B_PFULL), np & 1)) {
-          tc_fence_after();
-          // this CTA's value columns: atoms 4*half .. 4*half+3 of the stage
-          const uint64_t dv = desc_sw128_mn(
-              sb + OFF_C + (np % kStages) * kCBytes + 4 * half * kAtomBytes, kAtomBytes, 1024);
-#pragma unroll
-          for (int kk = 0; kk < kNT / 16; ++kk)
-#pragma unroll
-            for (int a = 0; a < 256 / kPvN; ++a)  // 64-column blocks are atoms kAtomBytes apart
-              mma_bf16(tmem + TM_O + kPvN * a, dp0 + (uint64_t)(kk * 2),
-                       dv + (uint64_t)(kk * 128 + a * (kPvN / 64) * (kAtomBytes >> 4)), IDESC_PV,
-                       (np > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar(B_PVDONE));
-          mma_commit(bar(B_VEMPTY + np % kStages));
-          ++np;
-          progressed = true;
-        } else if (nb < na && mbar_test(bar(B_VFULL + nb % kStages), (nb / kStages) & 1)) {
+        auto qkb_go = [&] {
+          return nb < na && mbar_test(bar(B_VFULL + nb % kStages), (nb / kStages) & 1);
+        };
+        auto pv_go = [&] { return np < nb && mbar_test(bar(B_PFULL), np & 1); };
+        auto qka_go = [&] {
+          return na == nb && na < ntiles &&
+                 mbar_test(bar(B_AFULL + na % kStages), (na / kStages) & 1) &&
+                 mbar_test(bar(B_SEMPTY), (na & 1) ^ 1);
+        };
+        auto do_qkb = [&] {
           fence_async_smem();  // rows written by cp.async (generic proxy)
           tc_fence_after();
           const uint64_t db = desc_sw128(sb + OFF_C + (nb % kStages) * kCBytes, 1024);
@@ -577,9 +568,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(bar(B_SFULL));
           ++nb;
           progressed = true;
-        } else if (na == nb && na < ntiles &&
-                   mbar_test(bar(B_AFULL + na % kStages), (na / kStages) & 1) &&
-                   mbar_test(bar(B_SEMPTY), (na & 1) ^ 1)) {
+        };
+        auto do_pv = [&] {
+          tc_fence_after();
+          // this CTA's value columns: atoms 4*half .. 4*half+3 of the stage
+          const uint64_t dv = desc_sw128_mn(
+              sb + OFF_C + (np % kStages) * kCBytes + 4 * half * kAtomBytes, kAtomBytes, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kNT / 16; ++kk)
+#pragma unroll
+            for (int a = 0; a < 256 / kPvN; ++a)  // 64-column blocks are atoms kAtomBytes apart
+              mma_bf16(tmem + TM_O + kPvN * a, dp0 + (uint64_t)(kk * 2),
+                       dv + (uint64_t)(kk * 128 + a * (kPvN / 64) * (kAtomBytes >> 4)), IDESC_PV,
+                       (np > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(B_PVDONE));
+          mma_commit(bar(B_VEMPTY + np % kStages));
+          ++np;
+          progressed = true;
+        };
+        auto do_qka = [&] {
           fence_async_smem();  // rows written by cp.async (generic proxy)
           tc_fence_after();
           const uint64_t db = desc_sw128(sb + OFF_C + (na % kStages) * kCBytes, 1024);
@@ -600,6 +607,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(bar(B_AEMPTY + na % kStages));
           ++na;
           progressed = true;
+        };
+        // bf16 cache: QK-B first; e4m3 cache: PV first (its value atoms come
+        // from the producers, behind group A)
+        if constexpr (FP8) {
+          if (pv_go()) do_pv();
+          else if (qkb_go()) do_qkb();
+          else if (qka_go()) do_qka();
+        } else {
+          if (qkb_go()) do_qkb();
+          else if (pv_go()) do_pv();
+          else if (qka_go()) do_qka();
         }
         if (progressed) {
           t0 = clock64();
@@ -657,12 +675,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_QREADY));  // the staged atoms are read: the stages are free
     }
+    // bf16 cache: group V of tile m (this CTA's value atoms, 2048 chunks, 8 per
+    // thread), once PV(m-2) has freed the stage and the producers have
+    // published m's indices.  Tile m+1's goes out in tile m's iteration right
+    // after the wait for PV(m-1), the release of its stage, which that
+    // iteration waits for anyway before storing P(m).  The producers thus only
+    // fetch group A, and the copies are issued by 15 warps instead of 7
+    // (probe: 27 against 20 B/cycle per SM).  For an e4m3 cache the producers
+    // fetch both groups.
+    auto fetch_v = [&](int m) -> bool {
+      if constexpr (FP8) {
+        return true;
+      } else {
+        const int st = m % kStages, ring = m % kIdxRing;
+        const bool w = mbar_wait(bar(B_VEMPTY + st), ((m / kStages) & 1) ^ 1, R.status) &&
+                       mbar_wait(bar(B_IDX + ring), (m / kIdxRing) & 1, R.status);
+        if (w) {
+#pragma unroll
+          for (int j = 0; j < kChunksV / kSoftmaxThreads; ++j)
+            issue(st, ring, (tid - kSoftmax0) + kSoftmaxThreads * j, false);
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
+                         bar(B_VFULL + st))
+                     : "memory");
+        return w;
+      }
+    };
+    static_assert(kChunksV % kSoftmaxThreads == 0, "group V split");
+    // tile 0's value atoms go where the staged query was: after every
+    // softmax thread has read it
+    if constexpr (!FP8) {
+      if (ntiles > 0 && !(mbar_wait(bar(B_QREADY), 0, R.status) && fetch_v(0))) *abort_flag = 1;
+    }
     // row h of P: this warpgroup's 32 rows are 16-byte chunks 4wg .. 4wg+3
     uint8_t* const prow = smem + OFF_P + h * 128;
     float m2 = -INFINITY, l = 0.f;
     bool ok = true;
     for (int n = 0; ok && n < ntiles; ++n) {
-      const int st = n % kStages;
       float s[32];
       // S(n) retired; then the tile's validity bits and scales are visible
       // (B_IDX: the producers published them; they cannot publish tile
@@ -703,6 +752,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P of tile n-1 is consumed and O is final up to tile n-1 once PV(n-1) retired
       const bool t_ok = n == 0 || __all_sync(0xffffffffu,
                                              mbar_wait(bar(B_PVDONE), (n - 1) & 1, R.status));
+      if constexpr (!FP8) {
+        if (n + 1 < ntiles && !fetch_v(n + 1)) *abort_flag = 1;
+      }
       if (mt > m2 + kRescale || (m2 == -INFINITY && mt != -INFINITY)) {
         const float m_new = fmaxf(mt, m2);
         const float alpha = ex2(m2 - m_new);  // 0 when m2 = -inf
@@ -746,6 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_PFULL));
     }
     if (!ok) *abort_flag = 1;
+    asm volatile("cp.async.wait_all;" ::: "memory");
     // combine the two warpgroups' denominators (the first barrier retires the
     // last tile's reads of the half maxima)
     asm volatile("bar.sync 1, 256;" ::: "memory");
