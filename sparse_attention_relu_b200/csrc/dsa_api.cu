@@ -235,7 +235,7 @@ dsa_status_t check_host(const Rows& R, const dsa_forward_args_t* h, const dsa_fo
 // that has not completed is released by the runtime once it completes; waits
 // already enqueued on it are unaffected).
 struct CallEvents {
-  cudaEvent_t e[4] = {};
+  cudaEvent_t e[5] = {};
   bool ok = true;
   CallEvents() {
     for (auto& x : e)
@@ -491,7 +491,8 @@ dsa_status_t dsa_forward_host(const dsa_layout_t* layout, const dsa_forward_args
   if ((s = copy_streams(&hs, &ds))) return s;
   CallEvents ev;
   if (!ev.ok) return DSA_ERR_CUDA;
-  const cudaEvent_t start = ev.e[0], in = ev.e[1], done = ev.e[2], end = ev.e[3];
+  const cudaEvent_t start = ev.e[0], in = ev.e[1], done = ev.e[2], end = ev.e[3],
+                    in_q = ev.e[4];
   // bytes of one row of each array
   const size_t esz = a->idx_dtype == DSA_F32 ? 4 : a->idx_dtype == DSA_BF16 ? 2 : 1;
   const size_t qi_row = (size_t)a->H_I * a->D_I * esz, hv_row = (size_t)a->H_I * 4,
@@ -518,12 +519,14 @@ dsa_status_t dsa_forward_host(const dsa_layout_t* layout, const dsa_forward_args
   for (int32_t r0 = 0; ok && r0 < R.n_q; r0 += p.slab) {
     const int32_t nr = (R.n_q - r0) < p.slab ? (R.n_q - r0) : p.slab;
     const size_t r = (size_t)r0, n = (size_t)nr;
-    // slab i's query rows go up while slab i-1 computes and slab i-2's results come down
+    // slab i's query rows go up while slab i-1 computes and slab i-2's results come down;
+    // the indexer's inputs first, under their own event, so that the indexer and the
+    // top-k run while the attention's (larger) queries are still on the way
     ok = copy(a->q_idx, host->q_idx, r * qi_row, n * qi_row, hs) &&
          copy(a->q_scale, host->q_scale, r * hv_row, n * hv_row, hs) &&
-         copy(a->w, host->w, r * hv_row, n * hv_row, hs) &&
-         copy(a->q, host->q, r * q_row, n * q_row, hs) && cudaEventRecord(in, hs) == cudaSuccess &&
-         cudaStreamWaitEvent(st, in, 0) == cudaSuccess;
+         copy(a->w, host->w, r * hv_row, n * hv_row, hs) && cudaEventRecord(in, hs) == cudaSuccess &&
+         copy(a->q, host->q, r * q_row, n * q_row, hs) &&
+         cudaEventRecord(in_q, hs) == cudaSuccess && cudaStreamWaitEvent(st, in, 0) == cudaSuccess;
     if (!ok) break;
     if (p.fused) {
       if ((s = launch_indexer_select(R, r0, nr, a->idx_dtype, a->H_I, a->D_I, a->q_idx,
@@ -535,6 +538,10 @@ dsa_status_t dsa_forward_host(const dsa_layout_t* layout, const dsa_forward_args
                            a->k_idx, a->k_scale, scores, false, st)))
         break;
       if ((s = launch_topk(R, r0, nr, scores, R.max_len, a->k, idx, st))) break;
+    }
+    if (cudaStreamWaitEvent(st, in_q, 0) != cudaSuccess) {
+      ok = false;
+      break;
     }
     if ((s = run_attn(R, r0, nr, a->q, a->kv, a->kv_scale, idx, a->k, a->H, a->D_K, a->D_V,
                       a->sm_scale,
