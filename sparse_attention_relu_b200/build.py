@@ -1,6 +1,10 @@
 """Builds libdsa.so in-tree from csrc/*.cu for sm_100a (nvcc, no JIT cache).
 
-    python -m sparse_attention_relu_b200.build [--force]
+    python -m sparse_attention_relu_b200.build [--force] [--trace]
+
+--trace also builds libdsa_trace.so, a diagnostic copy whose attention kernel
+records per-tile clock64 stamps (attn_tc.cu compiled with -DDSA_ATTN_TRACE;
+stage_bench.py --trace reads them).  The product path never loads it.
 """
 from __future__ import annotations
 
@@ -14,6 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libdsa.so")
+TRACE_LIB = os.path.join(HERE, "libdsa_trace.so")
 OBJ_DIR = os.path.join(HERE, "_build")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -37,9 +42,9 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def _compile(src: str) -> str:
-    obj = os.path.join(OBJ_DIR, os.path.basename(src) + ".o")
-    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+def _compile(src: str, extra=(), obj_dir: str = OBJ_DIR) -> str:
+    obj = os.path.join(obj_dir, os.path.basename(src) + ".o")
+    cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
@@ -64,5 +69,28 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_trace(verbose: bool = False) -> str:
+    """libdsa.so's objects with attn_tc.cu recompiled under -DDSA_ATTN_TRACE."""
+    if os.path.exists(TRACE_LIB) and up_to_date() and all(
+            os.path.getmtime(p) <= os.path.getmtime(TRACE_LIB) for p in _deps()):
+        return TRACE_LIB
+    attn = os.path.join(CSRC, "attn_tc.cu")
+    others = [os.path.join(OBJ_DIR, os.path.basename(s) + ".o") for s in _sources() if s != attn]
+    build(force=not all(os.path.exists(o) for o in others))
+    tdir = os.path.join(OBJ_DIR, "trace")
+    os.makedirs(tdir, exist_ok=True)
+    objs = [_compile(attn, ["-DDSA_ATTN_TRACE"], tdir)] + others
+    tmp = TRACE_LIB + f".tmp{os.getpid()}"
+    r = subprocess.run([NVCC, *ARCH, "-shared", "-o", tmp, *objs], capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+    os.replace(tmp, TRACE_LIB)
+    if verbose:
+        print("built", TRACE_LIB)
+    return TRACE_LIB
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True)
+    if "--trace" in sys.argv:
+        build_trace(verbose=True)

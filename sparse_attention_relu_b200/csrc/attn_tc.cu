@@ -229,6 +229,27 @@ __device__ __forceinline__ void store_codes(uint8_t* rowp, int c, int row, const
   *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (row & 7)) << 4)) = b;
 }
 
+// Diagnostic build only (-DDSA_ATTN_TRACE, libdsa_trace.so; stage_bench.py
+// --trace prints the table): clock64 stamps of each tile's events on the two
+// CTAs of one row -- the MMA thread's issue of each work item, the softmax
+// thread's waits, producer thread 0's copies.  The product library compiles
+// the stamps to nothing.
+#ifdef DSA_ATTN_TRACE
+constexpr int kTraceTiles = 64, kTraceEvents = 16;
+__device__ long long g_attn_trace[2 * kTraceTiles * kTraceEvents];
+__device__ long long g_attn_trace_t0[2];
+__device__ int g_attn_trace_item = -1;
+#define DSA_STAMP(n, f)                                                                \
+  do {                                                                                 \
+    if (tslot >= 0 && (n) >= 0 && (n) < kTraceTiles)                                   \
+      g_attn_trace[(tslot * kTraceTiles + (n)) * kTraceEvents + (f)] = clock64();      \
+  } while (0)
+#else
+#define DSA_STAMP(n, f) \
+  do {                  \
+  } while (0)
+#endif
+
 struct Split {
   int nsplit, tiles_per_split;
 };
@@ -298,6 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int half = blockIdx.x & 1;  // this CTA's output columns 256*half ..
+#ifdef DSA_ATTN_TRACE
+  const int tslot = (int)(blockIdx.x >> 1) == g_attn_trace_item ? half : -1;
+  if (threadIdx.x == 0 && tslot >= 0) g_attn_trace_t0[tslot] = clock64();
+#endif
   const int item = blockIdx.x >> 1;
   const int32_t rloc = item / sp.nsplit, split = item % sp.nsplit;
   const int32_t r = row0 + rloc;
@@ -482,6 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // first tile, once the staged query has left the stages)
         bool ok = (n > 0 || mbar_wait(bar(B_QREADY), 0, R.status)) &&
                   mbar_wait(bar(B_AEMPTY + st), par, R.status) && !*abort_flag;
+        if (tid == 0) DSA_STAMP(n, 10);
         if (!bar_and<2, kProducers>(ok)) {
           *abort_flag = 1;
           break;
@@ -493,6 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
                          bar(B_AFULL + st))
                      : "memory");
+        if (tid == 0) DSA_STAMP(n, 11);
         // (group V, this CTA's value columns, is fetched by the softmax
         // threads once PV(n-2) has released it)
       }
@@ -554,6 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : mbar_test(bar(B_SEMPTY), (na & 1) ^ 1) && mbar_test(afull, apar);
         };
         auto do_qkb = [&] {
+          DSA_STAMP(nb, 2);
           fence_async_smem();  // rows written by cp.async (generic proxy)
           tc_fence_after();
           const uint64_t db = desc_sw128(sb + OFF_C + (nb % kStages) * kCBytes, 1024);
@@ -569,10 +597,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int sub = 0; sub < 4; ++sub) qk_step(db, a, sub, 1u);
           }
           mma_commit(bar(B_SFULL));
+          DSA_STAMP(nb, 3);
           ++nb;
           progressed = true;
         };
         auto do_pv = [&] {
+          DSA_STAMP(np, 4);
           tc_fence_after();
           // this CTA's value columns: atoms 4*half .. 4*half+3 of the stage
           const uint64_t dv = desc_sw128_mn(
@@ -586,10 +616,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                        (np > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(B_PVDONE));
           mma_commit(bar(B_VEMPTY + np % kStages));
+          DSA_STAMP(np, 5);
           ++np;
           progressed = true;
         };
         auto do_qka = [&] {
+          DSA_STAMP(na, 0);
           fence_async_smem();  // rows written by cp.async (generic proxy)
           tc_fence_after();
           const uint64_t db = desc_sw128(sb + OFF_C + (na % kStages) * kCBytes, 1024);
@@ -608,6 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 qk_step(db, a < 4 ? 4 + a : 8, sub, (a > 0 || sub > 0) ? 1u : 0u);
           }
           mma_commit(bar(B_AEMPTY + na % kStages));
+          DSA_STAMP(na, 1);
           ++na;
           progressed = true;
         };
@@ -716,6 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
                          bar(B_VFULL + st))
                      : "memory");
+        if (tid == kSoftmax0) DSA_STAMP(m, 12);
         return w;
       }
     };
@@ -740,6 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  mbar_wait(bar(B_IDX + n % kIdxRing), (n / kIdxRing) & 1,
                                            R.status) &&
                                  !*abort_flag);
+      if (tid == kSoftmax0) DSA_STAMP(n, 6);
       if (w_ok) {
         tc_fence_after();
         tmem_ld32(tmem + lane_off + TM_S + 32 * wg, s);
@@ -750,6 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const uint32_t bits = vmask[(n % kIdxRing) * 2 + wg];
       mbar_arrive(bar(B_SEMPTY));  // the MMA may overwrite the score tile
+      if (tid == kSoftmax0) DSA_STAMP(n, 7);
       // this warpgroup's 32 rows of the tile: their cache scales (e4m3); the
       // ring entry stays until the producers refill it four tiles on
       const float* const tsc = ksc + (n % kIdxRing) * kNT + 32 * wg;
@@ -770,6 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P of tile n-1 is consumed and O is final up to tile n-1 once PV(n-1) retired
       const bool t_ok = n == 0 || __all_sync(0xffffffffu,
                                              mbar_wait(bar(B_PVDONE), (n - 1) & 1, R.status));
+      if (tid == kSoftmax0) DSA_STAMP(n, 8);
       if constexpr (!FP8) {
         if (n + 1 < ntiles && !fetch_v(n + 1)) *abort_flag = 1;
       }
@@ -814,6 +851,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();          // P stores before the PV MMA reads them
       tc_fence_before();           // a rescale's TMEM stores before the PV MMA
       mbar_arrive(bar(B_PFULL));
+      if (tid == kSoftmax0) DSA_STAMP(n, 9);
     }
     if (!ok) *abort_flag = 1;
     asm volatile("cp.async.wait_all;" ::: "memory");
@@ -988,3 +1026,17 @@ dsa_status_t launch_attn_tc_static(const Rows& R, int32_t row0, int32_t nrows, c
 }
 
 }  // namespace dsa
+
+#ifdef DSA_ATTN_TRACE
+// Diagnostic build only: selects the traced row (grid item, -1: none) and
+// copies the stamps out ([2][64][16] then the two CTA start stamps).
+extern "C" int dsa_attn_trace_select(int item) {
+  return (int)cudaMemcpyToSymbol(dsa::g_attn_trace_item, &item, sizeof(int));
+}
+extern "C" int dsa_attn_trace_copy(long long* host) {
+  int e = (int)cudaMemcpyFromSymbol(host, dsa::g_attn_trace, sizeof(dsa::g_attn_trace));
+  if (e) return e;
+  return (int)cudaMemcpyFromSymbol(host + 2 * dsa::kTraceTiles * dsa::kTraceEvents,
+                                   dsa::g_attn_trace_t0, sizeof(dsa::g_attn_trace_t0));
+}
+#endif

@@ -9,6 +9,14 @@ Small, fixed cases meant for profiler captures of a single kernel:
   attn/decode    64 sequences x 16384 tokens (cache from HBM), k scattered positions
   indexer|topk   e4m3 prefill of T tokens (the unit calls write full score rows)
 Prints one line with the last repetition's time and throughput.
+
+    python stage_bench.py --stage attn --case prefill --trace [--trace-row 3000]
+
+runs attn/prefill on libdsa_trace.so (built on demand: the attention kernel
+with per-tile clock64 stamps) and prints, for the two CTAs of one query row,
+the steady-state cycles between the events of a tile (medians over the middle
+tiles): the MMA thread's issue of QK-A, QK-B and PV, the softmax thread's
+waits, producer thread 0's copies.
 """
 from __future__ import annotations
 
@@ -114,6 +122,59 @@ def indexer_topk(stage: str, reps: int, T: int, k: int = 2048):
         print(f"topk T={T}: ms={ms:.3f} score read GB/s={pairs * 4 / ms / 1e6:.1f}")
 
 
+# event fields of the trace build (attn_tc.cu, DSA_STAMP)
+_EV = {"qka_b": 0, "qka_e": 1, "qkb_b": 2, "qkb_e": 3, "pv_b": 4, "pv_e": 5, "s_seen": 6,
+       "s_free": 7, "pv_prev_done": 8, "p_pub": 9, "a_empty": 10, "a_issued": 11, "v_issued": 12}
+
+
+def trace_attn(T: int, row: int, k: int = 2048):
+    import ctypes
+
+    import numpy as np
+
+    from sparse_attention_relu_b200 import build as B
+
+    dsa.LIB_PATH = B.build_trace()
+    L = dsa.lib()
+    L.dsa_attn_trace_select.argtypes = [ctypes.c_int]
+    L.dsa_attn_trace_copy.argtypes = [ctypes.c_void_p]
+    assert L.dsa_attn_trace_select(row) == 0
+    attn("prefill", 2, T, k)
+    torch.cuda.synchronize()
+    tiles, nev = 64, 16
+    buf = np.zeros(2 * tiles * nev + 2, np.int64)
+    assert L.dsa_attn_trace_copy(buf.ctypes.data_as(ctypes.c_void_p)) == 0
+    st = buf[: 2 * tiles * nev].reshape(2, tiles, nev)
+    t0 = buf[2 * tiles * nev:]
+    e = _EV
+    rows = [
+        ("tile period (QK-A issue to the next)", lambda a, n: a[n + 1, e["qka_b"]] - a[n, e["qka_b"]]),
+        ("QK-A issue, 20 K steps", lambda a, n: a[n, e["qka_e"]] - a[n, e["qka_b"]]),
+        ("QK-A issued -> QK-B issue starts", lambda a, n: a[n, e["qkb_b"]] - a[n, e["qka_e"]]),
+        ("QK-B issue, 16 K steps", lambda a, n: a[n, e["qkb_e"]] - a[n, e["qkb_b"]]),
+        ("QK-B issued -> softmax sees S", lambda a, n: a[n, e["s_seen"]] - a[n, e["qkb_e"]]),
+        ("softmax: S seen -> read and released", lambda a, n: a[n, e["s_free"]] - a[n, e["s_seen"]]),
+        ("S released -> next QK-A issue starts", lambda a, n: a[n + 1, e["qka_b"]] - a[n, e["s_free"]]),
+        ("softmax: released -> PV(n-1) retired", lambda a, n: a[n, e["pv_prev_done"]] - a[n, e["s_free"]]),
+        ("softmax: PV(n-1) retired -> P(n) published", lambda a, n: a[n, e["p_pub"]] - a[n, e["pv_prev_done"]]),
+        ("P(n) published -> PV(n) issue starts", lambda a, n: a[n, e["pv_b"]] - a[n, e["p_pub"]]),
+        ("PV issue, 4 K steps", lambda a, n: a[n, e["pv_e"]] - a[n, e["pv_b"]]),
+        ("producers: stage free -> group A issued", lambda a, n: a[n, e["a_issued"]] - a[n, e["a_empty"]]),
+    ]
+    for c in range(2):
+        a = st[c]
+        nt = int(np.count_nonzero(a[:, e["qka_b"]]))
+        if nt < 12:
+            print(f"CTA {c}: {nt} tiles traced, too few")
+            continue
+        mid = range(4, nt - 4)
+        print(f"row {row}, CTA {c} (output columns {256 * c}..{256 * c + 255}), {nt} tiles; "
+              f"first score tile seen {a[0, e['s_seen']] - t0[c]} cycles after the CTA starts")
+        for name, f in rows:
+            v = np.array([f(a, n) for n in mid])
+            print(f"  {name:44s} median {int(np.median(v)):6d}  min {int(v.min()):6d}  max {int(v.max()):6d}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--stage", choices=["attn", "indexer", "topk"], required=True)
@@ -121,8 +182,13 @@ def main():
     ap.add_argument("--reps", type=int, default=4)
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--kv", choices=["bf16", "e4m3"], default="bf16", help="MLA cache storage")
+    ap.add_argument("--trace", action="store_true",
+                    help="attn/prefill on the trace build: per-tile event table of one row")
+    ap.add_argument("--trace-row", type=int, default=3000)
     a = ap.parse_args()
-    if a.stage == "attn":
+    if a.trace:
+        trace_attn(a.tokens or 4096, a.trace_row)
+    elif a.stage == "attn":
         attn(a.case, a.reps, a.tokens or 4096, kv_dtype=a.kv)
     else:
         indexer_topk(a.stage, a.reps, a.tokens or 16384)
