@@ -37,6 +37,19 @@ def test_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), name
 
 
+def test_trace_entry_points_only_in_the_diagnostic_build(lib):
+    """The per-tile trace of the attention kernel is a separate library
+    (attn_tc.cu under -DDSA_ATTN_TRACE); the product library has none of it."""
+    from sparse_attention_relu_b200 import build
+
+    for name in ("dsa_attn_trace_select", "dsa_attn_trace_copy"):
+        assert not hasattr(lib, name), name
+    trace = ctypes.CDLL(build.build_trace())
+    for name in ("dsa_attn_trace_select", "dsa_attn_trace_copy"):
+        assert hasattr(trace, name), name
+    assert os.path.realpath(build.TRACE_LIB) != os.path.realpath(dsa.LIB_PATH)
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert dsa.dsa_status_string(s) and dsa.dsa_status_string(s) != "unknown status"
