@@ -243,6 +243,11 @@ size_t dsa_forward_workspace_size(const dsa_layout_t* layout, const dsa_forward_
  * of fp32 scores at max_len per row (4096 rows at 64K context).
  *  out [n_q, H, D_V] bf16; lse [n_q, H] fp32 or NULL;
  *  idx_out [n_q, k] int32 or NULL (then the indices live in the workspace).
+ * Decode with the environment variable DSA_FUSED_DECODE_SELECT set to "1" at
+ * the call runs the indexer with the top-k fused in (per-row candidate lists
+ * against a running threshold, no score rows; the same indices as the
+ * separate kernels).  Off by default: it is slower.  The workspace size
+ * depends on it, so query dsa_forward_workspace_size under the same setting.
  */
 dsa_status_t dsa_forward(const dsa_layout_t* layout, const dsa_forward_args_t* args, void* out,
                          float* lse, int32_t* idx_out, void* workspace, size_t ws_bytes,

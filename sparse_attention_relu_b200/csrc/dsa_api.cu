@@ -1,6 +1,7 @@
 // C ABI of libdsa: argument validation and the orchestration of the stages.
 // The semantics of each call are documented in include/dsa.h.
 #include <math.h>
+#include <stdlib.h>
 
 #include <mutex>
 
@@ -164,9 +165,15 @@ int32_t slab_rows(const Rows& R) {
   return (int32_t)rows;
 }
 
-// The fused decode selection is built and tested but not yet faster than the
-// separate top-k kernel, so dsa_forward does not take it.
-constexpr bool kFusedDecodeSelect = false;
+// The fused decode selection (indexer and top-k in one kernel, no score rows)
+// is built and tested but not yet faster than the separate top-k kernel, so
+// dsa_forward takes it only when the environment variable
+// DSA_FUSED_DECODE_SELECT is 1 at the call (and at the workspace query: the
+// two plans differ in size).
+bool fused_decode_select() {
+  const char* v = getenv("DSA_FUSED_DECODE_SELECT");
+  return v && v[0] == '1' && v[1] == 0;
+}
 
 struct ForwardPlan {
   int32_t slab;
@@ -182,7 +189,8 @@ ForwardPlan plan_forward(const Rows& R, const dsa_forward_args_t* a, bool own_id
   ForwardPlan p{};
   p.slab = slab_rows(R);
   if (slab_cap > 0 && slab_cap < p.slab) p.slab = slab_cap;
-  p.fused = kFusedDecodeSelect && indexer_select_supported(R, a->idx_dtype, a->H_I, a->D_I, a->k);
+  p.fused = fused_decode_select() &&
+            indexer_select_supported(R, a->idx_dtype, a->H_I, a->D_I, a->k);
   size_t o = 0;
   p.off_scores = o;
   o = align_up(o + (p.fused ? indexer_select_workspace(R, p.slab)

@@ -50,6 +50,32 @@ def test_trace_entry_points_only_in_the_diagnostic_build(lib):
     assert os.path.realpath(build.TRACE_LIB) != os.path.realpath(dsa.LIB_PATH)
 
 
+def test_fused_decode_selection_is_opt_in(lib, monkeypatch):
+    """dsa_forward plans the fused decode indexer + selection (candidate lists
+    instead of a score slab) only with DSA_FUSED_DECODE_SELECT=1; prefill
+    never takes it."""
+    P = 4096  # fake device addresses: the size query dereferences nothing
+    d = dict(idx_dtype=dsa.DSA_BF16, H_I=64, D_I=128, q_idx=P, q_scale=None, w=P, k_idx=P,
+             k_scale=None, H=128, D_K=576, D_V=512, sm_scale=0.1, q=P, kv=P, k=2048,
+             kv_dtype=dsa.DSA_BF16, kv_scale=None)
+    a = dsa.dsa_forward_args_t(*d.values())
+    lib.dsa_forward_workspace_size.restype = ctypes.c_size_t
+
+    def size(mode, env):
+        if env is None:
+            monkeypatch.delenv("DSA_FUSED_DECODE_SELECT", raising=False)
+        else:
+            monkeypatch.setenv("DSA_FUSED_DECODE_SELECT", env)
+        L = _layout(mode=mode, batch=4, max_len=4096, n_q=4 if mode == dsa.DSA_DECODE else 4096,
+                    n_k=4 * 4096)
+        return lib.dsa_forward_workspace_size(ctypes.byref(L), ctypes.byref(a))
+
+    off = size(dsa.DSA_DECODE, None)
+    assert off > 0 and size(dsa.DSA_DECODE, "0") == off and size(dsa.DSA_DECODE, "11") == off
+    assert size(dsa.DSA_DECODE, "1") != off
+    assert size(dsa.DSA_PREFILL, "1") == size(dsa.DSA_PREFILL, None)
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert dsa.dsa_status_string(s) and dsa.dsa_status_string(s) != "unknown status"

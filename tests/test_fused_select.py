@@ -1,7 +1,8 @@
 """The decode path's fused indexer + top-k against the unit calls and the oracle.
 
-dsa_forward in decode mode runs the indexer with the selection fused in: no
-score row is written; each score is kept as a candidate only when it reaches
+With DSA_FUSED_DECODE_SELECT=1 (off by default: not yet faster than the two
+kernels), dsa_forward in decode mode runs the indexer with the selection fused
+in: no score row is written; each score is kept as a candidate only when it reaches
 the row's running threshold (the k-th best counted so far), and the CTA that
 finishes a row selects its k best from the candidates ("GLM sparse
 attention", threshold figure).  The scores themselves are computed by the
@@ -19,6 +20,11 @@ import workloads
 from dsa_testutil import Dev
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _fused(monkeypatch):
+    monkeypatch.setenv("DSA_FUSED_DECODE_SELECT", "1")
 
 
 def _fused_vs_unit(dev):
