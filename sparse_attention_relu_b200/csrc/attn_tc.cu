@@ -252,6 +252,7 @@ __device__ int g_attn_trace_item = -1;
 
 struct Split {
   int nsplit, tiles_per_split;
+  int packed;  // the row's valid indices come first, at most t + 1 of them
 };
 
 // Fixed scratch for callers that cannot allocate device memory (see
@@ -328,7 +329,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int32_t r = row0 + rloc;
   const RowInfo ri = row_info(R, r);
   const int slot_lo = split * sp.tiles_per_split * kNT;
-  const int slot_hi = min(k, slot_lo + sp.tiles_per_split * kNT);
+  // (packed indices: the slots after min(t + 1, k) are all empty)
+  const int slot_end = sp.packed ? min(k, max(ri.t + 1, 0)) : k;
+  const int slot_hi = min(slot_end, slot_lo + sp.tiles_per_split * kNT);
   const int ntiles = slot_hi > slot_lo ? (slot_hi - slot_lo + kNT - 1) / kNT : 0;
 
   if (tid == 0) {
@@ -966,9 +969,10 @@ size_t attn_tc_workspace(int32_t nrows, int k, int H, int D_V) {
 dsa_status_t launch_attn_tc(const Rows& R, int32_t row0, int32_t nrows, const uint16_t* q,
                             const void* kv, const float* kv_scale, const int32_t* idx, int k,
                             float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
-                            cudaStream_t st) {
+                            cudaStream_t st, bool packed) {
   if (nrows <= 0) return DSA_OK;
-  const Split sp = plan_split(nrows, k);
+  Split sp = plan_split(nrows, k);
+  sp.packed = packed ? 1 : 0;
   float *part_o = nullptr, *part_lse = nullptr;
   if (sp.nsplit > 1) {
     if (!ws || ws_bytes < attn_tc_workspace(nrows, k, kH, kDV)) return DSA_ERR_WORKSPACE;

@@ -139,13 +139,15 @@ size_t attn_ws(int32_t nrows, int k, int H, int D_K, int D_V) {
 }
 
 // kv_scale != NULL: an e4m3 cache with per-token scales, else bf16.
+// packed: idx is the chain's own top-k output (valid indices first, at most
+// t + 1 per row), whose empty trailing tiles the tensor-core kernel skips.
 dsa_status_t run_attn(const Rows& R, int32_t row0, int32_t nrows, const void* q, const void* kv,
                       const float* kv_scale, const int32_t* idx, int k, int H, int D_K, int D_V,
                       float sm_scale, void* out, float* lse, void* ws, size_t ws_bytes,
-                      cudaStream_t st) {
+                      cudaStream_t st, bool packed = false) {
   if (attn_tc_supported(H, D_K, D_V))
     return launch_attn_tc(R, row0, nrows, (const uint16_t*)q, kv, kv_scale, idx, k, sm_scale,
-                          (uint16_t*)out, lse, ws, ws_bytes, st);
+                          (uint16_t*)out, lse, ws, ws_bytes, st, packed);
   return launch_attn_simt(R, row0, nrows, (const uint16_t*)q, kv, kv_scale, idx, k, H, D_K, D_V,
                           sm_scale, (uint16_t*)out, lse, st);
 }
@@ -451,9 +453,10 @@ dsa_status_t dsa_forward_timed(const dsa_layout_t* layout, const dsa_forward_arg
       if ((s = launch_topk(R, r0, nr, scores, R.max_len, a->k, idx, st))) return s;
       if ((s = mark(1))) return s;
     }
+    // (idx is this chain's own top-k output: packed)
     if ((s = run_attn(R, r0, nr, a->q, a->kv, a->kv_scale, idx, a->k, a->H, a->D_K, a->D_V,
                       a->sm_scale, out,
-                      lse, ws + p.off_attn, p.total - p.off_attn, st)))
+                      lse, ws + p.off_attn, p.total - p.off_attn, st, true)))
       return s;
     if ((s = mark(2))) return s;
   }
@@ -553,7 +556,7 @@ dsa_status_t dsa_forward_host(const dsa_layout_t* layout, const dsa_forward_args
     }
     if ((s = run_attn(R, r0, nr, a->q, a->kv, a->kv_scale, idx, a->k, a->H, a->D_K, a->D_V,
                       a->sm_scale,
-                      dev_out, dev_lse, ws + p.off_attn, p.total - p.off_attn, st)))
+                      dev_out, dev_lse, ws + p.off_attn, p.total - p.off_attn, st, true)))
       break;
     ok = cudaEventRecord(done, st) == cudaSuccess &&
          cudaStreamWaitEvent(ds, done, 0) == cudaSuccess &&

@@ -56,10 +56,13 @@ dsa_status_t launch_attn_simt(const Rows& R, int32_t row0, int32_t nrows, const 
 // bf16 cache, or (kv_scale != NULL) e4m3 codes with one fp32 scale per token.
 bool attn_tc_supported(int H, int D_K, int D_V);
 size_t attn_tc_workspace(int32_t nrows, int k, int H, int D_V);
+// packed: each row's valid indices come first and number at most t + 1 (the
+// top-k's output), so the tiles after slot min(t + 1, k) hold no index and are
+// skipped; otherwise every one of the k slots is scanned.
 dsa_status_t launch_attn_tc(const Rows& R, int32_t row0, int32_t nrows, const uint16_t* q,
                             const void* kv, const float* kv_scale, const int32_t* idx, int k,
                             float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
-                            cudaStream_t st);
+                            cudaStream_t st, bool packed = false);
 
 // As launch_attn_tc, with the split partials in a fixed static device array
 // (DSA_ERR_WORKSPACE when the call needs more than it holds).
