@@ -452,9 +452,36 @@ def measured_traffic(kernel, cfg):
     return rec["bytes_per_launch"]
 
 
+STAGE_NAMES = {0: "indexer", 1: "topk", 2: "sparse_mla_attn", 3: "split_combine"}
+
+
+def stage_roof(wl, kind, peaks):
+    """The roofline of one stage on workload wl: its algorithmic work per
+    step (all rows), the bound that applies (tensor or HBM), the unit and the
+    peak.  None for a stage with no work of its own (the split merge)."""
+    w = algorithmic_work(wl)
+    c = wl.cfg
+    if kind == 2:
+        if c.mode == "decode":  # gather-bound: HBM roofline of the gathered rows
+            return w["attn_bytes"].sum(), "hbm", "GB/s", peaks["hbm"]
+        return w["attn_flop"].sum(), "tensor", "TFLOP/s", peaks["bf16_sustained"]
+    if kind == 0:
+        if c.mode == "decode":
+            return w["idx_bytes"].sum(), "hbm", "GB/s", peaks["hbm"]
+        return (w["idx_flop"].sum(), "tensor", "TFLOP/s",
+                peaks["bf16_sustained"] * (2.0 if c.idx_dtype == "e4m3" else 1.0))
+    if kind == 1:
+        return w["topk_bytes"].sum(), "hbm", "GB/s", peaks["hbm"]
+    return None
+
+
+def _rate(work, ms, unit):
+    """work per ms in the unit's scale (TFLOP/s or GB/s)."""
+    return work / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
+
+
 def roofline(wl, stage_ms, peaks):
     """Dominant kernel (largest share of the step) against its roofline."""
-    w = algorithmic_work(wl)
     tot = {k: sum(v) for k, v in stage_ms.items()}
     if not tot:
         return None, {}
@@ -463,41 +490,38 @@ def roofline(wl, stage_ms, peaks):
     c = wl.cfg
     slabs = math.ceil(wl.n_q / slab_rows(wl))
     # every launch of a kind processes one slab; average work per launch
-    if kind == 2:
-        work = w["attn_flop"].sum() / slabs
-        bound, unit = "tensor", "TFLOP/s"
-        achieved = work / (per_launch_ms * 1e-3) / 1e12
-        peak = peaks["bf16_sustained"]
-        if c.mode == "decode":  # gather-bound: HBM roofline of the gathered rows
-            work = w["attn_bytes"].sum() / slabs
-            bound, unit = "hbm", "GB/s"
-            achieved = work / (per_launch_ms * 1e-3) / 1e9
-            peak = peaks["hbm"]
-    elif kind == 0:
-        if c.mode == "decode":
-            work = w["idx_bytes"].sum() / slabs
-            bound, unit = "hbm", "GB/s"
-            achieved = work / (per_launch_ms * 1e-3) / 1e9
-            peak = peaks["hbm"]
-        else:
-            work = w["idx_flop"].sum() / slabs
-            bound, unit = "tensor", "TFLOP/s"
-            achieved = work / (per_launch_ms * 1e-3) / 1e12
-            peak = peaks["bf16_sustained"] * (2.0 if c.idx_dtype == "e4m3" else 1.0)
-    else:
-        work = w["topk_bytes"].sum() / slabs
-        bound, unit = "hbm", "GB/s"
-        achieved = work / (per_launch_ms * 1e-3) / 1e9
-        peak = peaks["hbm"]
-    names = {0: "indexer", 1: "topk", 2: "sparse_mla_attn", 3: "split_combine"}
-    shares = {names[k]: round(v / sum(tot.values()), 4) for k, v in tot.items()}
-    return {"kernel": names[kind], "bound": bound, "achieved": round(achieved, 2),
+    work, bound, unit, peak = stage_roof(wl, kind, peaks)
+    work /= slabs
+    achieved = _rate(work, per_launch_ms, unit)
+    shares = {STAGE_NAMES[k]: round(v / sum(tot.values()), 4) for k, v in tot.items()}
+    return {"kernel": STAGE_NAMES[kind], "bound": bound, "achieved": round(achieved, 2),
             "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
-            "traffic": measured_traffic(names[kind], c),
+            "traffic": measured_traffic(STAGE_NAMES[kind], c),
             "peak_source": peaks["source"] + (" (x2 nominal fp8/bf16 ratio)" if
                                              unit == "TFLOP/s" and kind == 0 and
                                              c.idx_dtype == "e4m3" else ""),
             "launch_ms": round(per_launch_ms, 4)}, shares
+
+
+def stage_rooflines(wl, stage_ms, steps, ms_per_step, peaks):
+    """Every stage against its roofline, and the step's roofline fraction:
+    the sum of the stages' roofline times (algorithmic work / peak) over the
+    measured step time.  stage_ms holds the launches of `steps` timed steps."""
+    stages, bound_ms = {}, 0.0
+    for kind, launches in sorted(stage_ms.items()):
+        r = stage_roof(wl, kind, peaks)
+        if r is None or not launches:
+            continue
+        work, bound, unit, peak = r
+        ms = sum(launches) / steps  # this stage's device time per step
+        achieved = _rate(work, ms, unit)
+        floor_ms = work / (peak * (1e12 if unit == "TFLOP/s" else 1e9)) * 1e3
+        bound_ms += floor_ms
+        stages[STAGE_NAMES[kind]] = {"bound": bound, "unit": unit, "achieved": round(achieved, 2),
+                                     "peak": peak, "frac": round(achieved / peak, 4),
+                                     "ms_per_step": round(ms, 4),
+                                     "roofline_ms": round(floor_ms, 4)}
+    return stages, (round(bound_ms / ms_per_step, 4) if ms_per_step > 0 else None)
 
 
 # --------------------------------------------------------------- ranks
@@ -675,6 +699,8 @@ def main():
             "roofline": roof, "stage_share": shares,
             "gpu_launches": launches,
         }
+        line["stage_roofline"], line["step_roofline_frac"] = stage_rooflines(
+            wl, stage_ms, a.steps, ms, peaks)
         if e2e:
             line["e2e"] = {"value": round(job_throughput(tokens, e2e_ms, world), 1), "unit": "tokens/s",
                            "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
@@ -692,6 +718,9 @@ def main():
                               "unit": "tokens/s", "ms_per_step": round(dms, 4),
                               "roofline": droof, "stage_share": dshares,
                               "gpu_launches": dec[3]}
+            (line["decode"]["stage_roofline"],
+             line["decode"]["step_roofline_frac"]) = stage_rooflines(dwl, dec[2], a.steps, dms,
+                                                                     peaks)
             if dec[5]:
                 line["decode"]["index_reuse"] = _reuse_line(dec[5], dreuse_ms, dwl.n_q, world)
             if dec[4]:
