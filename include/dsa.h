@@ -271,7 +271,9 @@ dsa_status_t dsa_forward_timed(const dsa_layout_t* layout, const dsa_forward_arg
  * query rows: slab i's query rows are copied up (on a copy stream of the
  * library's own) while slab i-1 computes on `stream` and slab i-2's output
  * is copied down (on a second copy stream), so the two PCIe directions and
- * the kernels overlap.  The kernels and their arguments are those of
+ * the kernels overlap.  A slab's indexer inputs (q_idx, q_scale, w) go up
+ * first, so its indexer and top-k start while its attention queries (q) are
+ * still on the way.  The kernels and their arguments are those of
  * dsa_forward, and so are the results, up to the rounding order of the
  * attention sums (the order of a row's selected indices is unspecified, as
  * for dsa_topk, so two calls of either entry point may differ in the last
